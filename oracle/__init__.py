@@ -1,0 +1,101 @@
+"""CPU oracle for fused MoE top-k gating -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product (``moe_router_gating_b200``)
+never does, and this package imports nothing from the product.
+
+The arithmetic lives in ``gating_oracle.c`` (plain C, fp64, full per-row sort),
+written from the naive three-step form on the chenxutan.com page, section 4.1
+"MoE Gating": logits = hidden @ gate_weight; top-k of the logits; softmax of
+the k selected values.  Every function of it is pinned by
+``tests/test_oracle_pins.py``; no part is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "gating_oracle.c")
+_LIB = os.path.join(_HERE, "libgating_oracle.so")
+GCC_FLAGS = ["-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off"]
+
+_lock = threading.Lock()
+_libs: dict = {}
+
+
+def compile_oracle(src: str, out: str) -> str:
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *GCC_FLAGS, src, "-o", tmp, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(SOURCE):
+        compile_oracle(SOURCE, _LIB)
+    return _LIB
+
+
+@dataclass
+class OracleResult:
+    scores: np.ndarray    # fp32 [T, k]
+    scores64: np.ndarray  # fp64 [T, k]
+    ids: np.ndarray       # int32 [T, k]
+    gap: np.ndarray       # fp64 [T]
+    logits: np.ndarray | None  # fp64 [T, E] when requested
+
+
+class Oracle:
+    """ctypes handle on one compiled copy of the oracle source."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        vp, i64 = ctypes.c_void_p, ctypes.c_int64
+        lib.oracle_fused_topk_gating.argtypes = [vp, vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp, vp]
+        lib.oracle_fused_topk_gating.restype = ctypes.c_int
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = ctypes.c_int
+        self._lib = lib
+
+    def max_threads(self) -> int:
+        return int(self._lib.oracle_max_threads())
+
+    def gating(self, hidden_bits: np.ndarray, gate_bits: np.ndarray, k: int,
+               want_logits: bool = False) -> OracleResult:
+        x = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+        w = np.ascontiguousarray(gate_bits, dtype=np.uint16)
+        T, H = x.shape
+        H2, E = w.shape
+        if H != H2:
+            raise ValueError(f"hidden is [T,{H}] but gate_weight is [{H2},E]")
+        scores = np.zeros((T, k), dtype=np.float32)
+        scores64 = np.zeros((T, k), dtype=np.float64)
+        ids = np.full((T, k), -1, dtype=np.int32)
+        gap = np.zeros(T, dtype=np.float64)
+        logits = np.zeros((T, E), dtype=np.float64) if want_logits else None
+        rc = self._lib.oracle_fused_topk_gating(
+            x.ctypes.data, w.ctypes.data, T, H, E, k, scores.ctypes.data, scores64.ctypes.data,
+            ids.ctypes.data, gap.ctypes.data, logits.ctypes.data if logits is not None else None)
+        if rc != 0:
+            raise ValueError(f"oracle_fused_topk_gating returned {rc} (T={T} H={H} E={E} k={k})")
+        return OracleResult(scores, scores64, ids, gap, logits)
+
+
+def load(lib_path: str | None = None) -> Oracle:
+    path = lib_path or build()
+    with _lock:
+        if path not in _libs:
+            _libs[path] = Oracle(path)
+        return _libs[path]
+
+
+def fused_topk_gating(hidden_bits: np.ndarray, gate_bits: np.ndarray, k: int,
+                      want_logits: bool = False) -> OracleResult:
+    """Oracle result for bf16-bit inputs ``hidden[T,H]`` and ``gate_weight[H,E]``."""
+    return load().gating(hidden_bits, gate_bits, k, want_logits)
