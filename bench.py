@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoE top-k gating operator on B200.
+
+One step = one fused gating call (logits -> top-k -> softmax, one kernel launch)
+over one batch of synthetic tokens.  Default workload: the training-microbatch
+router, T=65536 tokens, H=7168, E=256 experts, k=8 (hidden 940 MB > L2).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one process per GPU)
+every rank gates its own batch of T tokens (token shards, no collective on the
+data path: weak scaling); time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (the fp64 definition, as it stands)
+on this host's cores, on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "fused top-k gating tokens/s"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NVML_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+                0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="train", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (earlier measurement on this pool)"
+
+
+def workload_desc(wl):
+    extra = ""
+    if wl.kind == "skew":
+        extra = f", +3u shared direction, dominant {list(wl.dominant)}, duplicated pairs {list(wl.duplicate_pairs)}"
+    return (f"{wl.name}: T={wl.T} H={wl.H} E={wl.E} k={wl.k}; synthetic bf16 hidden ~N(0,1), "
+            f"gate ~N(0,1/H), seed {wl.seed}{extra}")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def time_oracle(wl, seconds: float):
+    """Oracle tokens/s on a bounded row sample of `wl` (rows from the start)."""
+    import oracle
+    orc = oracle.load()
+    w_bits = wl.gate_weight()
+    probe = min(wl.T, 32)
+    x = wl.hidden_rows(0, probe)
+    t0 = time.perf_counter()
+    orc.gating(x, w_bits, wl.k)
+    rate = probe / max(time.perf_counter() - t0, 1e-6)
+    rows = int(min(wl.T, max(probe, rate * seconds)))
+    x = wl.hidden_rows(0, rows)
+    t0 = time.perf_counter()
+    orc.gating(x, w_bits, wl.k)
+    dt = time.perf_counter() - t0
+    return rows / dt, rows, dt, orc.max_threads()
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    orc = oracle.load()
+    w_bits = wl.gate_weight()
+    total_steps = args.steps + args.warmup
+    per_step_s = max(0.05, min(2.0, 150.0 / max(total_steps, 1)))
+    probe = min(wl.T, 32)
+    t0 = time.perf_counter()
+    orc.gating(wl.hidden_rows(0, probe), w_bits, wl.k)
+    rate = probe / max(time.perf_counter() - t0, 1e-6)
+    rows = int(min(wl.T, max(1, rate * per_step_s)))
+    x = wl.hidden_rows(0, rows)
+    for _ in range(args.warmup):
+        orc.gating(x, w_bits, wl.k)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.gating(x, w_bits, wl.k)
+    dt = time.perf_counter() - t0
+    value = rows * args.steps / dt
+    sample = f"first {rows} of {wl.T} tokens per step (fp64 oracle, full sort), same gate"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
+                   "tokens_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.max_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, local_rank: int, period_s: float = 0.02):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            cvd = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ids = [s.strip() for s in cvd.split(",") if s.strip()]
+            if ids and local_rank < len(ids):
+                tok = ids[local_rank]
+                h = (pynvml.nvmlDeviceGetHandleByIndex(int(tok)) if tok.isdigit()
+                     else pynvml.nvmlDeviceGetHandleByUUID(tok))
+            else:
+                h = pynvml.nvmlDeviceGetHandleByIndex(local_rank)
+            self._nvml, self._h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception as e:  # no NVML: report clocks as unavailable
+            self._nvml = None
+            self.error = repr(e)
+
+    def _run(self):
+        p, h = self._nvml, self._h
+        while not self._stop.is_set():
+            try:
+                sm = p.nvmlDeviceGetClockInfo(h, p.NVML_CLOCK_SM)
+                util = p.nvmlDeviceGetUtilizationRates(h).gpu
+                reasons = self._reasons(h)
+                power = p.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((sm, util, reasons, power))
+            except Exception as e:
+                self.error = repr(e)
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": f"NVML unavailable: {self.error}"}
+        loaded = [s for s in self.samples if s[1] > 0] or self.samples
+        reasons = set()
+        for s in loaded:
+            for bit, name in NVML_REASONS.items():
+                if s[2] & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {
+            "sm_mhz": statistics.median([s[0] for s in loaded]) if loaded else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": sorted(reasons),
+            "samples": len(self.samples),
+            "samples_under_load": len([s for s in self.samples if s[1] > 0]),
+            "power_w_max": max([s[3] for s in self.samples]) if self.samples else None,
+            "source": "NVML (same counters as nvidia-smi), sampled every 20 ms during the timed region",
+        }
+
+
+# ---------------------------------------------------------------------------
+def kernel_source_digest() -> str:
+    from moe_router_gating_b200 import build as tkbuild
+    h = hashlib.sha256()
+    for p in tkbuild._inputs():
+        if p.endswith(".py"):
+            continue
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(wl, digest: str):
+    """dram read+write bytes per launch from a committed ncu summary, if it was
+    taken on the current kernel sources (same digest); else None."""
+    path = os.path.join(PROFILE_DIR, f"traffic_{wl.name}.txt")
+    if not os.path.exists(path):
+        return None, None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if "=" in line and not line.lstrip().startswith("#"):
+                k, v = line.split("=", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_digest") != digest:
+        return None, f"{os.path.basename(path)} was taken on other kernel sources"
+    return float(vals["dram_bytes_per_launch"]), os.path.basename(path)
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import moe_router_gating_b200 as tk
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- inputs: seeded host arrays, each rank gates its own token shard ----
+    rank_wl = workloads.RouterWorkload(wl.name, wl.T, wl.H, wl.E, wl.k, wl.kind, wl.seed + rank,
+                                       wl.dominant, wl.duplicate_pairs)
+    x_bits = rank_wl.hidden()
+    w_bits = rank_wl.gate_weight()
+    x_host = workloads.to_torch_bf16(x_bits)
+    w = workloads.to_torch_bf16(w_bits).to(dev)
+    hidden_bytes = wl.T * wl.H * 2
+    big = hidden_bytes > L2_BYTES
+    x = x_host.to(dev)
+    scores = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    flush = None if big else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        tk.fused_topk_gating(x, w, wl.k, scores=scores, ids=ids, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    tk.device_error(clear=True)
+
+    sampler = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        if big:
+            # inputs larger than L2: back-to-back launches between two events
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for _ in range(args.steps):
+                step()
+            ev1.record(stream)
+            torch.cuda.synchronize(dev)
+            elapsed_ms = ev0.elapsed_time(ev1)
+            launch_ms = elapsed_ms / args.steps
+        else:
+            # small inputs: flush L2 (write 2x L2) between steps, time each launch alone
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                step()
+                b.record(stream)
+            torch.cuda.synchronize(dev)
+            per = [a.elapsed_time(b) for a, b in evs]
+            elapsed_ms = sum(per)
+            launch_ms = elapsed_ms / args.steps
+    torch.cuda.synchronize(dev)
+    barrier()
+    err = tk.device_error(clear=True)
+    if err:
+        raise SystemExit(f"device error word {err:#x}: a kernel wait expired during the timed region")
+
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_max_ms = float(t.item())
+    ms_per_step = elapsed_max_ms / args.steps
+    value = world * wl.T * args.steps / (elapsed_max_ms / 1e3)
+
+    # ---- end to end through the host-buffer C-ABI call (pinned host memory) ----
+    x_pinned = x_host.pin_memory()
+    s_host = torch.empty((wl.T, wl.k), dtype=torch.float32).pin_memory()
+    i_host = torch.empty((wl.T, wl.k), dtype=torch.int32).pin_memory()
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    for _ in range(2):
+        tk.fused_topk_gating_host(x_pinned, w, wl.k, s_host, i_host, x, scores, ids, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        tk.fused_topk_gating_host(x_pinned, w, wl.k, s_host, i_host, x, scores, ids, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * wl.T * e2e_steps / (float(te.item()) / 1e3)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    # ---- roofline of the (only) kernel ----
+    peaks, peak_src = load_peaks()
+    bytes_alg = wl.algorithmic_bytes()
+    flops = wl.flops()
+    t_s = launch_ms / 1e3
+    hbm_ach = bytes_alg / t_s / 1e9
+    tc_ach = flops / t_s / 1e12
+    t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    digest = kernel_source_digest()
+    traffic, traffic_src = profiled_traffic(wl, digest)
+    hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+           "frac": hbm_ach / peaks["hbm_gbs"], "traffic": traffic}
+    tc = {"bound": "tensor", "achieved": tc_ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+          "frac": tc_ach / peaks["bf16_tflops"], "traffic": traffic}
+    primary, secondary = (hbm, tc) if t_hbm >= t_tc else (tc, hbm)
+    roofline = dict(primary)
+    roofline.update({
+        "peak_source": f"{peak_src}; HBM = copy GB/s, tensor = cuBLAS bf16 burst TFLOP/s",
+        "roofline_frac": max(t_hbm, t_tc) / t_s,
+        "algorithmic_bytes_per_launch": bytes_alg, "flops_per_launch": flops,
+        "launch_ms": launch_ms, "traffic_source": traffic_src,
+        "kernel_source_digest": digest,
+        "secondary": {k: secondary[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
+    })
+
+    plan = tk.make_plan(wl.T, wl.H, wl.E, wl.k, torch.cuda.get_device_properties(dev).multi_processor_count)
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        v, rows, dt, cores = time_oracle(wl, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"first {rows} of {wl.T} tokens ({dt:.1f} s, fp64 oracle with full sort, all host threads)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": workload_desc(wl), "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
+            "tokens_per_rank_per_step": wl.T,
+            "arithmetic": "bf16 x bf16 products, fp32 accumulate (tcgen05), fp32 top-k and softmax",
+            "l2": ("inputs larger than L2: hidden is %.0f MB per step (gate %.2f MB stays L2-resident by design)"
+                   % (hidden_bytes / 1e6, wl.H * wl.E * 2 / 1e6)) if big else
+                  "L2 flushed (256 MB write) before every timed launch; each launch timed alone",
+            "parallelism": "single GPU" if world == 1 else f"{world} ranks, independent token shards, no collective",
+            "launch": plan,
+        },
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": hidden_bytes,
+                "d2h_bytes_per_step": wl.T * wl.k * 8,
+                "path": "tk_gating_fused_topk_host: pinned host hidden -> device, kernel, scores+ids -> pinned host"},
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    wl = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,162 @@
+/*
+ * tk_gating.h -- fused MoE top-k gating on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The operation (chenxutan.com, "TileKernels 深度解析", section 4.1 "MoE
+ * Gating"): the router's three-step naive form
+ *
+ *     logits          = hidden_states @ gate_weight        [T,H] x [H,E]
+ *     topk_vals, ids  = topk(logits, k)                     k largest per token
+ *     scores          = softmax(topk_vals) over the k values
+ *
+ * replaced by one kernel launch in which the logits never leave the chip
+ * (tensor memory and registers only; the page's "no write-back of
+ * intermediates to global memory").
+ *
+ * Semantics fixed by this library where the page is silent:
+ *   - logits accumulate in fp32 from bf16 inputs (no bf16 rounding of logits);
+ *   - ranking order is logit descending, then expert index ascending (equal
+ *     logits go to the lower expert index; -0 and +0 compare equal);
+ *   - ids[t, 0..k-1] are in rank order, scores[t, 0] >= scores[t, 1] >= ...;
+ *   - scores[t, j] = exp(v_j - v_0) / sum_i exp(v_i - v_0), fp32.
+ *
+ * Conventions for every entry point below:
+ *   - Pointers marked "device" are CUDA global-memory addresses on the current
+ *     device; the caller allocates and owns every buffer.  The library keeps no
+ *     per-call state and allocates no device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous: they return once the work is enqueued.  Launch
+ *     failures return TK_ERR_CUDA; faults inside a kernel surface at the
+ *     caller's next synchronisation.
+ *   - Invalid arguments are rejected before any CUDA call; nothing is written.
+ *   - There is no CPU fallback: without an sm_100 device every compute entry
+ *     point returns TK_ERR_UNSUPPORTED or TK_ERR_CUDA.
+ */
+#ifndef TK_GATING_H
+#define TK_GATING_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TK_API __attribute__((visibility("default")))
+#else
+#define TK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TK_OK = 0,
+  TK_ERR_INVALID_ARG = -1,    /* null pointer, negative size, k out of [1, E], ... */
+  TK_ERR_UNSUPPORTED = -2,    /* valid request outside what the kernels handle */
+  TK_ERR_ALIGNMENT = -3,      /* a pointer is not 16-byte aligned */
+  TK_ERR_CUDA = -4,           /* a CUDA runtime/driver call failed */
+  TK_ERR_DEVICE_TIMEOUT = -5  /* a kernel's bounded wait expired (device error word set) */
+} tk_status;
+
+/* Limits of the fused kernels. */
+#define TK_GATING_MAX_EXPERTS 256
+#define TK_GATING_MAX_TOPK 16
+
+/*
+ * tk_gating_fused_topk -- the fused gating operator.
+ *
+ *   hidden       device, bf16 [T, H] row-major (token t at hidden + t*H).
+ *   gate_weight  device, bf16 [H, E] row-major (the [H,E] orientation of
+ *                `hidden_states @ gate_weight`; expert e is column e).
+ *   T            tokens, T >= 0.  T == 0 returns TK_OK and launches nothing.
+ *   H            hidden size, H >= 8 and H % 8 == 0 (16-byte row pitch).
+ *   E            experts, 16 <= E <= 256 and E % 8 == 0.
+ *   k            experts kept per token, 1 <= k <= min(E, 16).
+ *   scores       device, out fp32 [T, k] row-major.
+ *   ids          device, out int32 [T, k] row-major.
+ *   stream       cudaStream_t (void*), may be NULL.
+ *
+ * Errors:
+ *   TK_ERR_INVALID_ARG   T < 0, H < 1, E < 1, k < 1, k > E, or a null pointer
+ *                        when T > 0;
+ *   TK_ERR_UNSUPPORTED   H or E not a multiple of 8, E < 16, E > 256, k > 16,
+ *                        T >= 2^31 - 128, or the current device is not sm_100;
+ *   TK_ERR_ALIGNMENT     a pointer is not 16-byte aligned;
+ *   TK_ERR_CUDA          a CUDA call (device query, descriptor encode, launch)
+ *                        failed.
+ * Size checks come first, so an invalid size is reported even with null
+ * pointers; T == 0 with valid sizes returns TK_OK before pointers are looked at.
+ */
+TK_API tk_status tk_gating_fused_topk(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,
+                               int32_t k, float* scores, int32_t* ids, void* stream);
+
+/*
+ * tk_gating_fused_topk_host -- the same operator for inputs and outputs that
+ * live in host memory (an end-to-end call).  On `stream` it copies hidden from
+ * host to the caller's device staging buffer, runs the fused kernel, and copies
+ * scores and ids back to host.  The gate stays device-resident (model weights).
+ *
+ *   hidden_host  host, bf16 [T, H]; page-locked memory makes the copy async.
+ *   gate_weight  device, bf16 [H, E].
+ *   scores_host  host, out fp32 [T, k].   ids_host  host, out int32 [T, k].
+ *   hidden_dev   device staging, bf16 [T, H].
+ *   scores_dev   device staging, fp32 [T, k].   ids_dev  device staging, int32 [T, k].
+ *
+ * Host buffers must stay valid until the stream reaches this point.  Same
+ * errors as tk_gating_fused_topk, plus TK_ERR_INVALID_ARG for null host
+ * pointers.
+ */
+TK_API tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* gate_weight, int64_t T, int64_t H,
+                                    int64_t E, int32_t k, float* scores_host, int32_t* ids_host, void* hidden_dev,
+                                    float* scores_dev, int32_t* ids_dev, void* stream);
+
+/* Kernel variants chosen by the planner. */
+typedef enum {
+  TK_VARIANT_NONE = 0,        /* T == 0: nothing to launch */
+  TK_VARIANT_ROW_TILES = 1,   /* persistent: each CTA owns whole 128-token tiles */
+  TK_VARIANT_SPLIT_H = 2      /* a cluster of CTAs splits H for one tile, DSMEM reduction */
+} tk_variant;
+
+/* The launch the library makes for a problem (host logic, no GPU needed). */
+typedef struct {
+  int32_t variant;      /* tk_variant */
+  int32_t block_m;      /* tokens per tile */
+  int32_t n_pad;        /* MMA N: E rounded up to a multiple of 16 */
+  int32_t num_tiles;    /* ceil(T / block_m) */
+  int32_t k_blocks;     /* ceil(H / 64) */
+  int32_t split_h;      /* CTAs sharing one tile's H range (1 = none) */
+  int32_t stages;       /* shared-memory ring depth */
+  int32_t grid;         /* CTAs launched */
+  int32_t cluster;      /* CTAs per cluster */
+  int32_t threads;      /* threads per CTA */
+  int32_t smem_bytes;   /* dynamic shared memory per CTA */
+  int32_t tmem_cols;    /* tensor-memory columns allocated per CTA */
+} tk_gating_plan;
+
+/*
+ * tk_gating_make_plan -- fill *plan with the launch tk_gating_fused_topk makes
+ * for (T, H, E, k) on a device with `num_sms` SMs.  Validates like
+ * tk_gating_fused_topk (pointers excepted).  Makes no CUDA call.
+ */
+TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan);
+
+/*
+ * tk_gating_device_error -- read the device error word of the current device
+ * (bits set by kernels whose bounded waits expired; 0 = none) into *word, and
+ * clear it when `clear` is non-zero.  Synchronises the device.  Returns
+ * TK_ERR_DEVICE_TIMEOUT when the word is non-zero, TK_OK otherwise.
+ */
+TK_API tk_status tk_gating_device_error(uint32_t* word, int32_t clear);
+
+/*
+ * tk_gating_set_wait_timeout_ns -- limit (nanoseconds) of every bounded wait in
+ * the kernels launched afterwards from this process (default 1e9).  Values
+ * below 1000 are rejected with TK_ERR_INVALID_ARG.
+ */
+TK_API tk_status tk_gating_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/* Static string for a status code. */
+TK_API const char* tk_gating_status_string(tk_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TK_GATING_H */

@@ -1,0 +1,161 @@
+"""ctypes marshalling for libtk_gating.so (argument checks and pointers only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_PKG)
+HEADER = os.path.join(_ROOT, "include", "tk_gating.h")
+_LIB_PATH = os.path.join(_PKG, "libtk_gating.so")
+
+TK_OK = 0
+TK_ERR_INVALID_ARG = -1
+TK_ERR_UNSUPPORTED = -2
+TK_ERR_ALIGNMENT = -3
+TK_ERR_CUDA = -4
+TK_ERR_DEVICE_TIMEOUT = -5
+
+_lock = threading.Lock()
+_lib = None
+
+
+class TkGatingError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+        self.status = status
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "variant", "block_m", "n_pad", "num_tiles", "k_blocks", "split_h", "stages", "grid", "cluster",
+        "threads", "smem_bytes", "tmem_cols")]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                                   "`python -m moe_router_gating_b200.build` (needs nvcc)")
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+            lib.tk_gating_fused_topk.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp]
+            lib.tk_gating_fused_topk.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_host.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp]
+            lib.tk_gating_fused_topk_host.restype = ctypes.c_int
+            lib.tk_gating_make_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(_Plan)]
+            lib.tk_gating_make_plan.restype = ctypes.c_int
+            lib.tk_gating_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+            lib.tk_gating_device_error.restype = ctypes.c_int
+            lib.tk_gating_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+            lib.tk_gating_set_wait_timeout_ns.restype = ctypes.c_int
+            lib.tk_gating_status_string.argtypes = [ctypes.c_int]
+            lib.tk_gating_status_string.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    """Function names declared in include/tk_gating.h."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*TK_API\s+(?:const\s+)?\w+\s*\*?\s*(tk_gating_\w+)\s*\(", text, re.M)))
+
+
+def status_string(status: int) -> str:
+    return library().tk_gating_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != TK_OK:
+        raise TkGatingError(status, where)
+
+
+def _stream_handle(stream, device) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream)
+
+
+def fused_topk_gating_ptr(hidden: int, gate_weight: int, T: int, H: int, E: int, k: int, scores: int, ids: int,
+                          stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the tk_status."""
+    return int(library().tk_gating_fused_topk(hidden, gate_weight, T, H, E, k, scores, ids, stream))
+
+
+def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, stream=None):
+    """``(scores[T,k] fp32, ids[T,k] int32) = softmax(topk(hidden @ gate_weight))``.
+
+    ``hidden`` is a CUDA bf16 ``[T, H]`` tensor and ``gate_weight`` a CUDA bf16
+    ``[H, E]`` tensor, both contiguous.  Output tensors may be passed in.  The
+    launch goes on ``stream`` (default: the current torch stream).
+    """
+    import torch
+    if hidden.dtype != torch.bfloat16 or gate_weight.dtype != torch.bfloat16:
+        raise TypeError("hidden and gate_weight must be torch.bfloat16")
+    if hidden.dim() != 2 or gate_weight.dim() != 2 or hidden.shape[1] != gate_weight.shape[0]:
+        raise ValueError(f"shapes {tuple(hidden.shape)} @ {tuple(gate_weight.shape)} do not chain")
+    if not hidden.is_cuda or not gate_weight.is_cuda or hidden.device != gate_weight.device:
+        raise ValueError("hidden and gate_weight must be CUDA tensors on one device")
+    if not hidden.is_contiguous() or not gate_weight.is_contiguous():
+        raise ValueError("hidden and gate_weight must be contiguous (row-major)")
+    T, H = hidden.shape
+    E = gate_weight.shape[1]
+    if scores is None:
+        scores = torch.empty((T, top_k), dtype=torch.float32, device=hidden.device)
+    if ids is None:
+        ids = torch.empty((T, top_k), dtype=torch.int32, device=hidden.device)
+    if scores.shape != (T, top_k) or ids.shape != (T, top_k) or scores.dtype != torch.float32 \
+            or ids.dtype != torch.int32 or not scores.is_contiguous() or not ids.is_contiguous():
+        raise ValueError("scores must be fp32 [T,k] and ids int32 [T,k], contiguous")
+    with torch.cuda.device(hidden.device):
+        st = library().tk_gating_fused_topk(hidden.data_ptr(), gate_weight.data_ptr(), T, H, E, int(top_k),
+                                            scores.data_ptr(), ids.data_ptr(),
+                                            _stream_handle(stream, hidden.device))
+    _check(st, "tk_gating_fused_topk")
+    return scores, ids
+
+
+def fused_topk_gating_host(hidden_host, gate_weight, top_k: int, scores_host, ids_host, hidden_dev, scores_dev,
+                           ids_dev, stream=None) -> None:
+    """End-to-end call: host ``hidden_host`` in, host ``scores_host``/``ids_host``
+    out, through caller-owned device staging tensors; asynchronous on ``stream``."""
+    T, H = hidden_host.shape
+    E = gate_weight.shape[1]
+    import torch
+    with torch.cuda.device(gate_weight.device):
+        st = library().tk_gating_fused_topk_host(
+            hidden_host.data_ptr(), gate_weight.data_ptr(), T, H, E, int(top_k), scores_host.data_ptr(),
+            ids_host.data_ptr(), hidden_dev.data_ptr(), scores_dev.data_ptr(), ids_dev.data_ptr(),
+            _stream_handle(stream, gate_weight.device))
+    _check(st, "tk_gating_fused_topk_host")
+
+
+def make_plan(T: int, H: int, E: int, k: int, num_sms: int = 148) -> dict:
+    """The launch the library would make (host logic only; no GPU needed)."""
+    p = _Plan()
+    st = library().tk_gating_make_plan(T, H, E, k, num_sms, ctypes.byref(p))
+    _check(st, "tk_gating_make_plan")
+    return {name: getattr(p, name) for name, _ in _Plan._fields_}
+
+
+def device_error(clear: bool = True) -> int:
+    """Device error word of the current device (0 = no kernel wait expired)."""
+    w = ctypes.c_uint32(0)
+    st = library().tk_gating_device_error(ctypes.byref(w), 1 if clear else 0)
+    if st not in (TK_OK, TK_ERR_DEVICE_TIMEOUT):
+        _check(st, "tk_gating_device_error")
+    return int(w.value)
+
+
+def set_wait_timeout_ns(timeout_ns: int) -> None:
+    _check(library().tk_gating_set_wait_timeout_ns(int(timeout_ns)), "tk_gating_set_wait_timeout_ns")

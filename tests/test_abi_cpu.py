@@ -1,0 +1,95 @@
+"""The C-ABI library on the host: loads, exports every declared symbol, and its
+host logic (validation, planning, status strings) behaves as the header says.
+No kernel is launched here."""
+import ctypes
+import subprocess
+
+import pytest
+import torch
+
+import moe_router_gating_b200 as tk
+from moe_router_gating_b200 import build as tkbuild
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    tkbuild.build()
+
+
+def test_exports_every_declared_symbol():
+    declared = tk.exported_symbols()
+    assert "tk_gating_fused_topk" in declared and len(declared) >= 6
+    lib = tk.library()
+    for name in declared:
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", tk.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert set(declared) <= exported, set(declared) - exported
+    # nothing else with C linkage leaks out under the library prefix
+    assert {s for s in exported if s.startswith("tk_")} == set(declared)
+
+
+def test_status_strings():
+    for code in (tk.TK_OK, tk.TK_ERR_INVALID_ARG, tk.TK_ERR_UNSUPPORTED, tk.TK_ERR_ALIGNMENT, tk.TK_ERR_CUDA,
+                 tk.TK_ERR_DEVICE_TIMEOUT):
+        assert tk.status_string(code).startswith("TK_")
+    assert tk.status_string(12345) == "unknown tk_status"
+
+
+@pytest.mark.parametrize("args,code", [
+    ((-1, 64, 16, 2), tk.TK_ERR_INVALID_ARG),       # negative T
+    ((8, 0, 16, 2), tk.TK_ERR_INVALID_ARG),         # H < 1
+    ((8, 64, 16, 0), tk.TK_ERR_INVALID_ARG),        # k < 1
+    ((8, 64, 16, 17), tk.TK_ERR_INVALID_ARG),       # k > E
+    ((8, 60, 16, 2), tk.TK_ERR_UNSUPPORTED),        # H % 8
+    ((8, 64, 20, 2), tk.TK_ERR_UNSUPPORTED),        # E % 8
+    ((8, 64, 8, 2), tk.TK_ERR_UNSUPPORTED),         # E < 16
+    ((8, 64, 264, 2), tk.TK_ERR_UNSUPPORTED),       # E > 256
+    ((8, 64, 64, 17), tk.TK_ERR_UNSUPPORTED),       # k > 16
+])
+def test_invalid_sizes_rejected_before_cuda(args, code):
+    T, H, E, k = args
+    assert tk.fused_topk_gating_ptr(16, 16, T, H, E, k, 16, 16) == code
+    with pytest.raises(tk.TkGatingError) as ei:
+        tk.make_plan(T, H, E, k)
+    assert ei.value.status == code
+
+
+def test_null_and_misaligned_pointers():
+    assert tk.fused_topk_gating_ptr(0, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_INVALID_ARG
+    assert tk.fused_topk_gating_ptr(16, 16, 8, 64, 16, 2, 0, 16) == tk.TK_ERR_INVALID_ARG
+    assert tk.fused_topk_gating_ptr(18, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_ALIGNMENT
+    assert tk.fused_topk_gating_ptr(16, 16, 8, 64, 16, 2, 16, 20) == tk.TK_ERR_ALIGNMENT
+
+
+def test_zero_tokens_is_a_no_op():
+    # T == 0: TK_OK without touching pointers or the device
+    assert tk.fused_topk_gating_ptr(0, 0, 0, 64, 16, 2, 0, 0) == tk.TK_OK
+    assert tk.make_plan(0, 64, 16, 2)["variant"] == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_no_cpu_fallback_without_gpu():
+    assert tk.fused_topk_gating_ptr(16, 16, 8, 64, 16, 2, 16, 16) in (tk.TK_ERR_CUDA, tk.TK_ERR_UNSUPPORTED)
+
+
+def test_plans_for_router_workloads():
+    import workloads
+    for wl in workloads.WORKLOADS.values():
+        p = tk.make_plan(wl.T, wl.H, wl.E, wl.k, 148)
+        assert p["variant"] in (1, 2)
+        assert p["n_pad"] % 16 == 0 and p["n_pad"] >= wl.E
+        assert p["smem_bytes"] <= 232448
+        assert p["tmem_cols"] in (32, 64, 128, 256, 512)
+        assert p["grid"] >= 1 and p["grid"] % max(p["cluster"], 1) == 0
+        assert p["stages"] >= 2
+        if p["variant"] == 1:
+            assert p["grid"] == min(p["num_tiles"], 148)
+
+
+def test_plan_tmem_and_smem_budget():
+    for E in range(16, 257, 8):
+        p = tk.make_plan(1000, 7168, E, min(8, E), 148)
+        assert p["tmem_cols"] >= 2 * ((p["n_pad"] + 31) // 32 * 32)
+        assert p["smem_bytes"] <= 232448

@@ -1,0 +1,163 @@
+"""CUDA path vs the CPU oracle, element by element, on seeded inputs.
+
+Rule (tests/parity.py): ids bit-exact on rows whose oracle gap between the
+k-th and (k+1)-th logit exceeds 2e-3 (order may differ only between adjacent
+ranks within 2e-3), selected logits within 2e-3 of the k-th elsewhere, scores
+within 1e-3 absolute, and exact ties resolved to the lower expert index.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_router_gating_b200 as tk
+import oracle
+import parity
+import workloads
+from gpu_helpers import check_against_oracle, check_workload, run_gpu, to_device_bf16
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def clean_error_word():
+    assert torch.cuda.is_available()
+    tk.device_error(clear=True)
+    yield
+    assert tk.device_error(clear=True) == 0, "a kernel wait expired during the GPU tests"
+
+
+def test_hand_worked_example_on_gpu():
+    g = json.load(open(os.path.join(GOLDEN, "hand_worked_2token.json")))
+    # pad H to 8 and E to 16 with zeros: the two tokens' top-2 and scores are unchanged
+    x = np.zeros((2, 8)); x[:, :2] = g["hidden"]
+    w = np.zeros((8, 16)); w[:2, :4] = g["gate_weight"]
+    s, i = run_gpu(workloads.round_bf16(x), workloads.round_bf16(w), 2)
+    assert i.tolist() == g["expected"]["ids"]
+    s0 = 1.0 / (1.0 + np.exp(-0.5))
+    assert np.allclose(s, [[s0, 1 - s0], [0.5, 0.5]], atol=1e-6, rtol=0)
+
+
+def test_tiny_workload():
+    check_workload(workloads.TINY)
+
+
+def test_deepseek_workload():
+    check_workload(workloads.DEEPSEEK)
+
+
+def test_skew_tie_workload():
+    info = check_workload(workloads.SKEW)
+    assert info["rows"] == workloads.SKEW.T
+
+
+@pytest.mark.parametrize("T", workloads.DECODE_TS)
+def test_decode_workloads(T):
+    check_workload(workloads.RouterWorkload(f"decode_T{T}", T, 7168, 256, 8))
+
+
+def test_train_workload_sampled_rows():
+    """Full-size run (the launch the benchmark times); the oracle checks sampled rows."""
+    wl = workloads.TRAIN
+    x_bits = wl.hidden()
+    w_bits = wl.gate_weight()
+    s, i = run_gpu(x_bits, w_bits, wl.k)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([np.arange(0, 256), np.arange(wl.T - 256, wl.T),
+                                     rng.choice(wl.T, 768, replace=False)]))
+    ref = oracle.fused_topk_gating(x_bits[rows], w_bits, wl.k, want_logits=True)
+    parity.check(s, i, ref, rows=rows, label="train-sampled")
+    # properties that hold on every row
+    assert np.all((i >= 0) & (i < wl.E))
+    srt = np.sort(i, axis=1)
+    assert np.all(srt[:, 1:] != srt[:, :-1])
+    assert np.all(np.abs(s.astype(np.float64).sum(axis=1) - 1.0) <= 1e-5)
+    assert np.all(np.diff(s, axis=1) <= 0)
+
+
+@pytest.mark.parametrize("T,H,E,k", [
+    (1, 64, 16, 1), (127, 64, 16, 16), (129, 72, 24, 5), (300, 520, 40, 3), (1000, 256, 64, 8),
+    (257, 128, 200, 7), (640, 1024, 256, 16), (130, 8, 256, 8), (2500, 96, 136, 4), (5000, 512, 256, 2),
+])
+def test_ragged_shapes(T, H, E, k):
+    wl = workloads.RouterWorkload(f"shape_{T}_{H}_{E}_{k}", T, H, E, k, seed=3)
+    check_workload(wl)
+
+
+def test_zero_gate_gives_uniform_scores():
+    T, H, E, k = 300, 256, 64, 8
+    x = workloads.normal_bf16(5, 1, 0, T * H).reshape(T, H)
+    w = np.zeros((H, E), dtype=np.uint16)
+    s, i = run_gpu(x, w, k)
+    assert np.array_equal(i, np.tile(np.arange(k, dtype=np.int32), (T, 1)))
+    assert np.all(np.abs(s - 1.0 / k) <= 1e-7)
+
+
+def test_k_equals_E_full_softmax():
+    wl = workloads.RouterWorkload("kE", 200, 256, 16, 16, seed=9)
+    check_workload(wl)
+
+
+def test_duplicate_columns_everywhere():
+    wl = workloads.RouterWorkload("dups", 2048, 512, 64, 8, seed=11)
+    w = wl.gate_weight().copy()
+    pairs = tuple((a, a + 32) for a in range(0, 32, 3))
+    for a, b in pairs:
+        w[:, b] = w[:, a]
+    check_against_oracle(wl.hidden(), w, wl.k, duplicate_pairs=pairs, label="dups")
+
+
+def test_zero_tokens_writes_nothing():
+    w = torch.zeros((64, 16), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    s, i = tk.fused_topk_gating(x, w, 2)
+    torch.cuda.synchronize()
+    assert s.shape == (0, 2) and i.shape == (0, 2)
+
+
+def test_writes_stay_inside_outputs():
+    wl = workloads.RouterWorkload("guard", 333, 256, 64, 6, seed=2)
+    x = to_device_bf16(wl.hidden())
+    w = to_device_bf16(wl.gate_weight())
+    pad = 64
+    s_buf = torch.full((wl.T * wl.k + 2 * pad,), 7.0, dtype=torch.float32, device="cuda")
+    i_buf = torch.full((wl.T * wl.k + 2 * pad,), -7, dtype=torch.int32, device="cuda")
+    s = s_buf[pad:pad + wl.T * wl.k].view(wl.T, wl.k)
+    i = i_buf[pad:pad + wl.T * wl.k].view(wl.T, wl.k)
+    tk.fused_topk_gating(x, w, wl.k, scores=s, ids=i)
+    torch.cuda.synchronize()
+    assert torch.all(s_buf[:pad] == 7.0) and torch.all(s_buf[-pad:] == 7.0)
+    assert torch.all(i_buf[:pad] == -7) and torch.all(i_buf[-pad:] == -7)
+
+
+def test_side_stream_and_repeatability():
+    wl = workloads.RouterWorkload("stream", 1111, 1024, 256, 8, seed=4)
+    x = to_device_bf16(wl.hidden())
+    w = to_device_bf16(wl.gate_weight())
+    s0, i0 = tk.fused_topk_gating(x, w, wl.k)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        s1, i1 = tk.fused_topk_gating(x, w, wl.k, stream=side)
+    side.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(i0, i1) and torch.equal(s0, s1)
+
+
+def test_host_entry_point_matches_device_entry_point():
+    wl = workloads.RouterWorkload("host", 700, 512, 64, 6, seed=6)
+    xb = workloads.to_torch_bf16(wl.hidden()).pin_memory()
+    w = to_device_bf16(wl.gate_weight())
+    s_h = torch.empty((wl.T, wl.k), dtype=torch.float32).pin_memory()
+    i_h = torch.empty((wl.T, wl.k), dtype=torch.int32).pin_memory()
+    x_d = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    s_d = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    i_d = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    tk.fused_topk_gating_host(xb, w, wl.k, s_h, i_h, x_d, s_d, i_d)
+    torch.cuda.synchronize()
+    s_ref, i_ref = tk.fused_topk_gating(xb.cuda(), w, wl.k)
+    assert torch.equal(i_h, i_ref.cpu()) and torch.equal(s_h, s_ref.cpu())
