@@ -55,6 +55,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (profiling cases)")
     return ap.parse_args()
 
 
@@ -79,21 +80,20 @@ def workload_desc(wl):
 # CPU oracle timing (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
 def time_oracle(wl, seconds: float):
-    """Oracle tokens/s on a bounded row sample of `wl` (rows from the start)."""
+    """Oracle tokens/s on a bounded row sample of `wl` (rows from the start):
+    doubles the sample until one timed run takes at least `seconds`."""
     import oracle
     orc = oracle.load()
     w_bits = wl.gate_weight()
-    probe = min(wl.T, 32)
-    x = wl.hidden_rows(0, probe)
-    t0 = time.perf_counter()
-    orc.gating(x, w_bits, wl.k)
-    rate = probe / max(time.perf_counter() - t0, 1e-6)
-    rows = int(min(wl.T, max(probe, rate * seconds)))
-    x = wl.hidden_rows(0, rows)
-    t0 = time.perf_counter()
-    orc.gating(x, w_bits, wl.k)
-    dt = time.perf_counter() - t0
-    return rows / dt, rows, dt, orc.max_threads()
+    rows = min(wl.T, 64)
+    while True:
+        x = wl.hidden_rows(0, rows)
+        t0 = time.perf_counter()
+        orc.gating(x, w_bits, wl.k)
+        dt = time.perf_counter() - t0
+        if dt >= seconds or rows == wl.T:
+            return rows / dt, rows, dt, orc.max_threads()
+        rows = int(min(wl.T, max(rows * 2, rows * 1.2 * seconds / max(dt, 1e-6))))
 
 
 def run_reference(args, wl):
@@ -410,6 +410,8 @@ def run_ours(args, wl):
 def main():
     args = parse_args()
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        wl = wl.with_T(args.tokens)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

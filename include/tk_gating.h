@@ -111,7 +111,8 @@ TK_API tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* 
 typedef enum {
   TK_VARIANT_NONE = 0,        /* T == 0: nothing to launch */
   TK_VARIANT_ROW_TILES = 1,   /* persistent: each CTA owns whole 128-token tiles */
-  TK_VARIANT_SPLIT_H = 2      /* a cluster of CTAs splits H for one tile, DSMEM reduction */
+  TK_VARIANT_SPLIT_H = 2,     /* a cluster of CTAs splits H for one tile, DSMEM reduction */
+  TK_VARIANT_ROW_PAIRS = 3    /* persistent CTA pairs (tcgen05 cta_group::2), 256-token tiles */
 } tk_variant;
 
 /* The launch the library makes for a problem (host logic, no GPU needed). */

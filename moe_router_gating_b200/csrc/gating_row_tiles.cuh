@@ -1,19 +1,28 @@
-// Persistent fused gating kernel: each CTA owns whole 128-token tiles.
+// Persistent fused gating kernel over whole token tiles.
 //
-// Per tile: logits[128, E] = hidden[128 rows, H] x gate[H, E] on the tensor
-// cores (tcgen05.mma, bf16 in, fp32 accumulate in tensor memory), then per row
-// top-k + softmax in registers; only scores and ids reach global memory.
+// Per tile: logits[rows, E] = hidden[rows, H] x gate[H, E] on the tensor cores
+// (tcgen05.mma, bf16 in, fp32 accumulate in tensor memory), then per row top-k
+// and softmax in registers; only scores and ids reach global memory.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: streams 64-wide K slices of the hidden tile
-//               (K-major, 128-byte swizzle) and of the gate (MN-major,
-//               128-byte swizzle, 64-expert boxes) through an S-stage ring.
-//   warp 1      allocates tensor memory; one lane issues tcgen05.mma (4 per
-//               stage, K=16 each) and commits stage releases / tile completion.
-//   warps 2..5  epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (one token
-//               row per thread), keeps a running top-k, applies the softmax and
-//               stores.  The accumulator is double-buffered in tensor memory so
-//               the epilogue of tile i overlaps the MMAs of tile i+1.
+// CG = 1: one CTA per 128-token tile (M = 128, N = E rounded up to 16).
+// CG = 2: a CTA pair (cluster of 2) per 256-token tile, tcgen05 cta_group::2
+//   (M = 256, N = 128 or 256).  Each CTA stages its own 128 hidden rows and half
+//   of the gate columns; the leader (cluster rank 0) issues the MMAs, which read
+//   both CTAs' shared memory and write each CTA's 128 rows x N logits into its
+//   own tensor memory.  Per CTA this halves the gate bytes each tile pulls from
+//   L2 compared with CG = 1.
+//
+// Warp roles (192 threads per CTA):
+//   warp 0      TMA producer: 64-wide K slices of the hidden rows (K-major,
+//               128-byte swizzle) and of the gate (MN-major, 128-byte swizzle,
+//               64-expert boxes) through an S-stage shared-memory ring.
+//   warp 1      allocates tensor memory; in the (leader) CTA one lane issues
+//               tcgen05.mma (4 per stage, K = 16 each) and the commits that free
+//               ring stages and publish finished accumulators.
+//   warps 2..5  epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (one token row
+//               per thread), keeps a running top-k, applies the softmax and
+//               stores.  The accumulator is double-buffered in tensor memory, so
+//               the epilogue of one tile overlaps the MMAs of the next.
 #pragma once
 
 #include <cuda.h>
@@ -24,7 +33,7 @@
 
 namespace tkg {
 
-constexpr int BLOCK_M = 128;                            // tokens per tile = TMEM lanes
+constexpr int BLOCK_M = 128;                            // token rows per CTA = TMEM lanes
 constexpr int BLOCK_K = 64;                             // bf16 per 128-byte swizzle row
 constexpr int UMMA_K = 16;                              // K per tcgen05.mma (kind::f16)
 constexpr int A_STAGE_BYTES = BLOCK_M * BLOCK_K * 2;    // 16 KB hidden slice
@@ -35,12 +44,12 @@ constexpr int ROW_TILE_THREADS = 64 + NUM_EPI_WARPS * 32;
 
 struct RowTileParams {
   int32_t T, H, E, k;
-  int32_t n_pad;        // MMA N (E rounded up to 16)
+  int32_t n_pad;        // MMA N (CG=1: E rounded up to 16; CG=2: 128 or 256)
   int32_t acc_stride;   // TMEM columns between the two accumulator buffers
-  int32_t num_tiles;
+  int32_t num_tiles;    // tiles of BLOCK_M * CG rows
   int32_t k_blocks;
   int32_t stages;
-  int32_t b_boxes;      // ceil(n_pad / 64) gate boxes per stage
+  int32_t b_boxes;      // gate boxes per stage loaded by each CTA
   uint32_t tmem_cols;
   uint64_t timeout_ns;
   float* scores;
@@ -64,10 +73,26 @@ __device__ __forceinline__ uint64_t b_desc_k_slice(uint32_t b_stage_addr, int kk
   return smem_desc_sw128(b_stage_addr + kk * (UMMA_K / 8) * 1024, B_BOX_BYTES, 1024);
 }
 
+// Offer 32 consecutive logits (columns c0 .. c0+31) of this thread's row;
+// columns at or beyond E (MMA padding) are skipped.
 template <int KMAX>
+__device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (&r)[32], int c0, int E) {
+  if (c0 + 32 <= E) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) top.offer(__uint_as_float(r[j]), c0 + j);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (c0 + j < E) top.offer(__uint_as_float(r[j]), c0 + j);
+  }
+}
+
+template <int KMAX, int CG>
 __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     gating_row_tiles_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                             const RowTileParams p) {
+  static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
+  constexpr bool kPair = CG == 2;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align_1024(smem_dyn);
   uint8_t* sA = smem;
@@ -82,6 +107,10 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;  // 0 = the pair's MMA leader
+  const bool leader = rank == 0;
+  const int first_tile = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_step = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -90,7 +119,7 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], NUM_EPI_WARPS * 32);
+      mbar_init(&acc_empty[b], NUM_EPI_WARPS * CG);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -99,11 +128,22 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     tma_prefetch_desc(&map_w);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, p.tmem_cols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(tmem_holder, p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (kPair) {
+    // the peer's loads and arrivals target the leader's barriers: both initialised first
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  } else {
+    __syncthreads();
+  }
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -112,21 +152,31 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       // ---------------- TMA producer ----------------
       const uint64_t pol_x = l2_policy_evict_first();  // hidden: streamed once
       const uint64_t pol_w = l2_policy_evict_last();   // gate: re-read by every tile
-      const uint32_t stage_tx = A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES;
+      const uint32_t stage_tx = CG * (A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES);
+      const int b_col0 = static_cast<int>(rank) * p.b_boxes * B_BOX_N;  // this CTA's gate columns
       uint32_t stage = 0, phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < p.num_tiles; tile += tile_step) {
+        const int row0 = tile * (BLOCK_M * CG) + static_cast<int>(rank) * BLOCK_M;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER, p.err_word)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], stage_tx);
-          tma_load_2d(sA + stage * A_STAGE_BYTES, &map_x, &full[stage], kb * BLOCK_K, tile * BLOCK_M, pol_x);
-          for (int j = 0; j < p.b_boxes; ++j)
-            tma_load_2d(sB + (stage * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], j * B_BOX_N,
-                        kb * BLOCK_K, pol_w);
+          if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
+          if constexpr (kPair) {
+            const uint32_t bar = map_shared_rank(smem_u32(&full[stage]), 0);
+            tma_load_2d_pair(sA + stage * A_STAGE_BYTES, &map_x, bar, kb * BLOCK_K, row0, pol_x);
+            for (int j = 0; j < p.b_boxes; ++j)
+              tma_load_2d_pair(sB + (stage * p.b_boxes + j) * B_BOX_BYTES, &map_w, bar, b_col0 + j * B_BOX_N,
+                               kb * BLOCK_K, pol_w);
+          } else {
+            tma_load_2d(sA + stage * A_STAGE_BYTES, &map_x, &full[stage], kb * BLOCK_K, row0, pol_x);
+            for (int j = 0; j < p.b_boxes; ++j)
+              tma_load_2d(sB + (stage * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], b_col0 + j * B_BOX_N,
+                          kb * BLOCK_K, pol_w);
+          }
           ++issued;
           if (++stage == static_cast<uint32_t>(p.stages)) {
             stage = 0;
@@ -134,26 +184,30 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           }
         }
       }
-      // Every load this thread issued lands before the CTA may exit.
-      const int pending = issued < p.stages ? issued : p.stages;
-      for (int n = 0; n < pending; ++n) {
-        if (stage == 0) {
-          stage = p.stages - 1;
-          phase ^= 1;
-        } else {
-          --stage;
+      // Every load issued lands before the CTA may exit.  The leader's full
+      // barriers count both CTAs' bytes; the peer's loads are covered by the
+      // leader's drain and the closing cluster barrier.
+      if (leader) {
+        const int pending = issued < p.stages ? issued : p.stages;
+        for (int n = 0; n < pending; ++n) {
+          if (stage == 0) {
+            stage = p.stages - 1;
+            phase ^= 1;
+          } else {
+            --stage;
+          }
+          mbar_wait(&full[stage], phase, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
         }
-        mbar_wait(&full[stage], phase, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ---------------- MMA issuer ----------------
-      const uint32_t idesc = idesc_bf16_f32(BLOCK_M, p.n_pad, false, true);
+      const uint32_t idesc = idesc_bf16_f32(BLOCK_M * CG, p.n_pad, false, true);
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
+      for (int tile = first_tile; ok && tile < p.num_tiles; tile += tile_step, ++local) {
         const uint32_t buf = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) break;
@@ -168,18 +222,34 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * p.b_boxes * B_BOX_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
-            umma_bf16(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc, (kb | kk) != 0);
-          umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
+            if constexpr (kPair)
+              umma_bf16_pair(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc, (kb | kk) != 0);
+            else
+              umma_bf16(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc, (kb | kk) != 0);
+          }
+          // frees the stage (in both CTAs of a pair) once these MMAs have read it
+          if constexpr (kPair)
+            umma_commit_pair_multicast(&empty[stage], 0x3);
+          else
+            umma_commit(&empty[stage]);
           if (++stage == static_cast<uint32_t>(p.stages)) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) umma_commit(&acc_full[buf]);
+        if (ok) {
+          if constexpr (kPair)
+            umma_commit_pair_multicast(&acc_full[buf], 0x3);
+          else
+            umma_commit(&acc_full[buf]);
+        }
       }
-      // Every MMA this thread issued completes before tensor memory is freed.
-      umma_commit(drain);
+      // Every MMA issued completes before tensor memory is freed.
+      if constexpr (kPair)
+        umma_commit_pair(drain);
+      else
+        umma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
     }
     __syncwarp();
@@ -188,7 +258,7 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     const int quad = warp & 3;  // TMEM lanes this warp may access
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int local = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+    for (int tile = first_tile; tile < p.num_tiles; tile += tile_step, ++local) {
       const uint32_t buf = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       bool ok = mbar_wait(&acc_full[buf], acc_phase, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
@@ -198,32 +268,46 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       RowTopK<KMAX> top;
       top.reset();
       const uint32_t acc_addr = lane_base + buf * p.acc_stride;
-      for (int c0 = 0; c0 < p.n_pad; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_32(acc_addr + c0, r);
+      // 64 columns per round trip: two loads, one wait
+      for (int c0 = 0; c0 < p.E; c0 += 64) {
+        uint32_t r0[32], r1[32];
+        const bool second = c0 + 32 < p.E;  // warp-uniform
+        tmem_ld_32(acc_addr + c0, r0);
+        if (second) tmem_ld_32(acc_addr + c0 + 32, r1);
         tmem_ld_wait();
-        if (c0 + 32 <= p.E) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) top.offer(__uint_as_float(r[j]), c0 + j);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c0 + j < p.E) top.offer(__uint_as_float(r[j]), c0 + j);
-        }
+        offer_chunk(top, r0, c0, p.E);
+        if (second) offer_chunk(top, r1, c0 + 32, p.E);
       }
+      // the accumulator buffer may be overwritten once every epilogue warp of
+      // the pair has read it
       tc_fence_before_sync();
-      mbar_arrive(&acc_empty[buf]);  // accumulator buffer may be overwritten
+      __syncwarp();
+      if (lane == 0) {
+        if (kPair && !leader)
+          mbar_arrive_remote(map_shared_rank(smem_u32(&acc_empty[buf]), 0));
+        else
+          mbar_arrive(&acc_empty[buf]);
+      }
 
-      const int64_t row = static_cast<int64_t>(tile) * BLOCK_M + quad * 32 + lane;
+      const int64_t row = static_cast<int64_t>(tile) * (BLOCK_M * CG) + rank * BLOCK_M + quad * 32 + lane;
       if (row < p.T) top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
     }
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (kPair) {
+    // neither CTA frees its shared or tensor memory while the pair still uses it
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else
+      tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 

@@ -48,24 +48,28 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
     plan->variant = TK_VARIANT_NONE;
     return TK_OK;
   }
-  const int n_pad = round_up(static_cast<int>(E), 16);
+  const bool pair = E > 64;  // gate halves of >= 64 experts per CTA (128-byte swizzle blocks)
+  const int cg = pair ? 2 : 1;
+  const int n_pad = pair ? round_up(static_cast<int>(E), 128) : round_up(static_cast<int>(E), 16);
   const int acc_stride = round_up(n_pad, 32);
-  const int b_boxes = (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+  const int b_boxes = pair ? n_pad / 2 / tkg::B_BOX_N : (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES;
   int stages = (kMaxDynamicSmem - kSmemReserve) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return TK_ERR_UNSUPPORTED;
-  const int64_t tiles = (T + tkg::BLOCK_M - 1) / tkg::BLOCK_M;
+  const int64_t rows_per_tile = static_cast<int64_t>(tkg::BLOCK_M) * cg;
+  const int64_t tiles = (T + rows_per_tile - 1) / rows_per_tile;
+  const int64_t units = num_sms / cg;  // CTAs (or CTA pairs) resident at once
 
-  plan->variant = TK_VARIANT_ROW_TILES;
-  plan->block_m = tkg::BLOCK_M;
+  plan->variant = pair ? TK_VARIANT_ROW_PAIRS : TK_VARIANT_ROW_TILES;
+  plan->block_m = static_cast<int32_t>(rows_per_tile);
   plan->n_pad = n_pad;
   plan->num_tiles = static_cast<int32_t>(tiles);
   plan->k_blocks = static_cast<int32_t>((H + tkg::BLOCK_K - 1) / tkg::BLOCK_K);
   plan->split_h = 1;
   plan->stages = stages;
-  plan->grid = static_cast<int32_t>(tiles < num_sms ? tiles : num_sms);
-  plan->cluster = 1;
+  plan->grid = static_cast<int32_t>((tiles < units ? tiles : units) * cg);
+  plan->cluster = cg;
   plan->threads = tkg::ROW_TILE_THREADS;
   plan->smem_bytes = stages * stage_bytes + kSmemReserve;
   plan->tmem_cols = static_cast<int32_t>(pow2_at_least(2 * acc_stride));
@@ -122,19 +126,33 @@ uint32_t* device_error_word() {
   return static_cast<uint32_t*>(p);
 }
 
-template <int KMAX>
+template <int KMAX, int CG>
 tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mw,
                            const tkg::RowTileParams& prm, cudaStream_t stream) {
-  auto kernel = tkg::gating_row_tiles_kernel<KMAX>;
+  auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem_bytes) != cudaSuccess)
     return TK_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(pl.threads);
   cfg.dynamicSmemBytes = pl.smem_bytes;
   cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = CG > 1 ? 1 : 0;
   if (cudaLaunchKernelEx(&cfg, kernel, mx, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
   return TK_OK;
+}
+
+template <int KMAX>
+tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mw,
+                             const tkg::RowTileParams& prm, cudaStream_t stream) {
+  if (pl.variant == TK_VARIANT_ROW_PAIRS) return launch_row_tiles<KMAX, 2>(pl, mx, mw, prm, stream);
+  return launch_row_tiles<KMAX, 1>(pl, mx, mw, prm, stream);
 }
 
 tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int64_t H, int64_t E, int32_t k,
@@ -169,18 +187,19 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   prm.num_tiles = pl.num_tiles;
   prm.k_blocks = pl.k_blocks;
   prm.stages = pl.stages;
-  prm.b_boxes = (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+  prm.b_boxes = pl.variant == TK_VARIANT_ROW_PAIRS ? pl.n_pad / 2 / tkg::B_BOX_N
+                                                   : (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   prm.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
   prm.timeout_ns = g_timeout_ns;
   prm.scores = scores;
   prm.ids = ids;
   prm.err_word = err;
 
-  if (k <= 1) return launch_row_tiles<1>(pl, mx, mw, prm, stream);
-  if (k <= 2) return launch_row_tiles<2>(pl, mx, mw, prm, stream);
-  if (k <= 4) return launch_row_tiles<4>(pl, mx, mw, prm, stream);
-  if (k <= 8) return launch_row_tiles<8>(pl, mx, mw, prm, stream);
-  return launch_row_tiles<16>(pl, mx, mw, prm, stream);
+  if (k <= 1) return launch_row_variant<1>(pl, mx, mw, prm, stream);
+  if (k <= 2) return launch_row_variant<2>(pl, mx, mw, prm, stream);
+  if (k <= 4) return launch_row_variant<4>(pl, mx, mw, prm, stream);
+  if (k <= 8) return launch_row_variant<8>(pl, mx, mw, prm, stream);
+  return launch_row_variant<16>(pl, mx, mw, prm, stream);
 }
 
 }  // namespace

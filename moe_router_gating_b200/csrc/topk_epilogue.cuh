@@ -24,21 +24,23 @@ struct RowTopK {
   }
 
   // Offer (value, index); indices must arrive in increasing order.
+  //
+  // Branch-free sorted insertion: with c_j = (value beats slot j), the new slot
+  // j holds the old slot j when !c_j, the old slot j-1 when c_{j-1} (the list is
+  // sorted, so c_{j-1} implies c_j), and the offered pair otherwise.  All slot
+  // updates read the old list, so they are independent of one another, and no
+  // lane of a warp ever waits on another lane's insertion.
   __device__ __forceinline__ void offer(float value, int32_t index) {
-    if (value > v[KMAX - 1]) {
-      v[KMAX - 1] = value;
-      i[KMAX - 1] = index;
+    bool c[KMAX];
 #pragma unroll
-      for (int j = KMAX - 1; j > 0; --j) {
-        const bool up = v[j] > v[j - 1];
-        const float tv = v[j];
-        const int32_t ti = i[j];
-        v[j] = up ? v[j - 1] : v[j];
-        i[j] = up ? i[j - 1] : i[j];
-        v[j - 1] = up ? tv : v[j - 1];
-        i[j - 1] = up ? ti : i[j - 1];
-      }
+    for (int j = 0; j < KMAX; ++j) c[j] = value > v[j];
+#pragma unroll
+    for (int j = KMAX - 1; j > 0; --j) {
+      v[j] = c[j] ? (c[j - 1] ? v[j - 1] : value) : v[j];
+      i[j] = c[j] ? (c[j - 1] ? i[j - 1] : index) : i[j];
     }
+    v[0] = c[0] ? value : v[0];
+    i[0] = c[0] ? index : i[0];
   }
 
   // Offer a candidate whose index may be lower than ones already held (used when

@@ -78,14 +78,17 @@ def test_plans_for_router_workloads():
     import workloads
     for wl in workloads.WORKLOADS.values():
         p = tk.make_plan(wl.T, wl.H, wl.E, wl.k, 148)
-        assert p["variant"] in (1, 2)
+        assert p["variant"] in (1, 2, 3)
         assert p["n_pad"] % 16 == 0 and p["n_pad"] >= wl.E
         assert p["smem_bytes"] <= 232448
         assert p["tmem_cols"] in (32, 64, 128, 256, 512)
         assert p["grid"] >= 1 and p["grid"] % max(p["cluster"], 1) == 0
         assert p["stages"] >= 2
         if p["variant"] == 1:
-            assert p["grid"] == min(p["num_tiles"], 148)
+            assert p["grid"] == min(p["num_tiles"], 148) and p["cluster"] == 1
+        if p["variant"] == 3:
+            assert p["cluster"] == 2 and p["block_m"] == 256 and p["n_pad"] in (128, 256)
+            assert p["grid"] == 2 * min(p["num_tiles"], 74)
 
 
 def test_plan_tmem_and_smem_budget():
