@@ -117,10 +117,13 @@ def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, st
     if scores.shape != (T, top_k) or ids.shape != (T, top_k) or scores.dtype != torch.float32 \
             or ids.dtype != torch.int32 or not scores.is_contiguous() or not ids.is_contiguous():
         raise ValueError("scores must be fp32 [T,k] and ids int32 [T,k], contiguous")
-    with torch.cuda.device(hidden.device):
-        st = library().tk_gating_fused_topk(hidden.data_ptr(), gate_weight.data_ptr(), T, H, E, int(top_k),
-                                            scores.data_ptr(), ids.data_ptr(),
-                                            _stream_handle(stream, hidden.device))
+    lib = library()
+    args = (hidden.data_ptr(), gate_weight.data_ptr(), T, H, E, int(top_k), scores.data_ptr(), ids.data_ptr())
+    if hidden.device.index == torch.cuda.current_device():
+        st = lib.tk_gating_fused_topk(*args, _stream_handle(stream, hidden.device))
+    else:
+        with torch.cuda.device(hidden.device):
+            st = lib.tk_gating_fused_topk(*args, _stream_handle(stream, hidden.device))
     _check(st, "tk_gating_fused_topk")
     return scores, ids
 

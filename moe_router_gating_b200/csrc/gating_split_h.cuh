@@ -1,0 +1,280 @@
+// Fused gating for few tokens: a cluster of C CTAs shares one 128-token tile
+// and splits the hidden dimension H between its CTAs.
+//
+// With T <= a few thousand tokens there are too few 128-token tiles to occupy
+// the GPU (T = 1..128 is a single tile), while every tile still streams the whole
+// gate matrix (H x E).  Here CTA r of the cluster accumulates the logits over
+// its own slice of H on the tensor cores:
+//
+//   1. mainloop (as in the row-tile kernel, one tile, k-blocks [kb0, kb1)):
+//      partial_r[128, E] in tensor memory;
+//   2. cluster barrier: every CTA's ring is drained, so its shared memory can
+//      take the exchange;
+//   3. CTA r owns the tile rows t with t % C == r.  Every CTA pushes row t of its
+//      partial (tensor memory -> registers -> distributed shared memory stores)
+//      into slot [t / C][r] of the owner's staging area;
+//   4. cluster barrier: the staging areas are complete;
+//   5. each owned row is split into G column segments, one thread each: the
+//      thread adds the C partials of its segment from local shared memory in
+//      rank order 0..C-1 (so a logit does not depend on which CTA owns its
+//      row), keeps a top-k of the segment, and the G lists are merged with warp
+//      shuffles; then softmax and store.
+//
+// Nothing but scores and ids is written to global memory.
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+#include "gating_row_tiles.cuh"
+#include "sm100_ptx.cuh"
+#include "topk_epilogue.cuh"
+#include "topk_merge.cuh"
+
+namespace tkg {
+
+// Warps: 0 producer, 1 MMA, 2..5 push partial rows (TMEM lane quadrants), 6..7
+// join the reduction; all 8 reduce.
+constexpr int SPLIT_THREADS = 256;
+constexpr int SPLIT_WARPS = SPLIT_THREADS / 32;
+constexpr int PUSH_WARPS = 4;
+constexpr int PUSH_SCRATCH_STRIDE = 36;                            // floats per scratch row (bank spread)
+constexpr int PUSH_SCRATCH_BYTES = 32 * PUSH_SCRATCH_STRIDE * 4;   // one 32 x 32 chunk per push warp
+
+struct SplitHParams {
+  int32_t T, H, E, k;
+  int32_t n_pad;        // MMA N (E rounded up to 16)
+  int32_t num_tiles;    // 128-token tiles
+  int32_t k_blocks;     // ceil(H / 64)
+  int32_t stages;
+  int32_t b_boxes;
+  int32_t row_stride;   // floats per staged partial row (round_up(E, 32) + 4)
+  uint32_t tmem_cols;
+  uint64_t timeout_ns;
+  float* scores;
+  int32_t* ids;
+  uint32_t* err_word;
+};
+
+template <int KMAX, int C>
+__global__ void __launch_bounds__(SPLIT_THREADS, 1)
+    gating_split_h_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                          const SplitHParams p) {
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = align_1024(smem_dyn);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + p.stages * A_STAGE_BYTES;
+  float* staging = reinterpret_cast<float*>(smem);  // reuses the ring once every CTA's MMAs are done
+  float* scratch = reinterpret_cast<float*>(sB + p.stages * p.b_boxes * B_BOX_BYTES);  // after the ring
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scratch) + PUSH_WARPS * PUSH_SCRATCH_BYTES);
+  uint64_t* empty = full + p.stages;
+  uint64_t* acc_full = empty + p.stages;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t r = cluster_ctarank();
+  const int tile = static_cast<int>(blockIdx.x / C);
+  // balanced split of the k-blocks; non-empty for every CTA since C <= k_blocks
+  const int kb0 = static_cast<int>((static_cast<int64_t>(r) * p.k_blocks) / C);
+  const int kb1 = static_cast<int>((static_cast<int64_t>(r + 1) * p.k_blocks) / C);
+  const int valid_rows = min(BLOCK_M, p.T - tile * BLOCK_M);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&map_x);
+    tma_prefetch_desc(&map_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer: this CTA's H slice of one tile ----------------
+      const uint64_t pol_x = l2_policy_evict_first();
+      const uint64_t pol_w = l2_policy_evict_last();
+      const uint32_t stage_tx = A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES;
+      uint32_t stage = 0, phase = 0;
+      int issued = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER, p.err_word)) break;
+        mbar_arrive_expect_tx(&full[stage], stage_tx);
+        tma_load_2d(sA + stage * A_STAGE_BYTES, &map_x, &full[stage], kb * BLOCK_K, tile * BLOCK_M, pol_x);
+        for (int j = 0; j < p.b_boxes; ++j)
+          tma_load_2d(sB + (stage * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], j * B_BOX_N, kb * BLOCK_K,
+                      pol_w);
+        ++issued;
+        if (++stage == static_cast<uint32_t>(p.stages)) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      const int pending = issued < p.stages ? issued : p.stages;
+      for (int n = 0; n < pending; ++n) {
+        if (stage == 0) {
+          stage = p.stages - 1;
+          phase ^= 1;
+        } else {
+          --stage;
+        }
+        mbar_wait(&full[stage], phase, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      const uint32_t idesc = idesc_bf16_f32(BLOCK_M, p.n_pad, false, true);
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
+        const uint32_t b_addr = smem_u32(sB + stage * p.b_boxes * B_BOX_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
+          umma_bf16(tmem_base, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc, (kb != kb0) | kk);
+        umma_commit(&empty[stage]);
+        if (++stage == static_cast<uint32_t>(p.stages)) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (ok) umma_commit(acc_full);
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
+    }
+    __syncwarp();
+  }
+
+  // Epilogue warps wait for this CTA's accumulator; then all rings of the
+  // cluster are idle and may be overwritten by the exchange.
+  const bool push_warp = warp >= 2 && warp < 2 + PUSH_WARPS;
+  bool acc_ok = true;
+  if (push_warp) {
+    acc_ok = mbar_wait(acc_full, 0, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
+    acc_ok = __all_sync(0xffffffffu, acc_ok);
+  }
+  tc_fence_before_sync();
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  tc_fence_after_sync();
+
+  // ---------------- push partial rows to their owners ----------------
+  // Each 32-row x 32-column chunk (row per thread from tensor memory) is
+  // transposed through this warp's scratch so that every remote store writes 128
+  // contiguous bytes of one row: 8 lanes per row, 4 rows per store instruction.
+  if (push_warp) {
+    const int quad = warp & 3;
+    if (acc_ok && quad * 32 < valid_rows) {
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+      float* my_scratch = scratch + (warp - 2) * (PUSH_SCRATCH_BYTES / 4);
+      const int sub_row = lane >> 3;       // 0..3: row within a group of 4
+      const int col4 = (lane & 7) * 4;     // column offset within the chunk
+      // 64 columns per tensor-memory round trip, pushed as two 32-column chunks
+      for (int c0 = 0; c0 < p.E; c0 += 64) {
+        uint32_t v[2][32];
+        const bool second = c0 + 32 < p.E;  // warp-uniform
+        tmem_ld_32(lane_base + c0, v[0]);
+        if (second) tmem_ld_32(lane_base + c0 + 32, v[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !second) break;
+          const int cc = c0 + 32 * h;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(my_scratch + lane * PUSH_SCRATCH_STRIDE + j) =
+                make_float4(__uint_as_float(v[h][j]), __uint_as_float(v[h][j + 1]), __uint_as_float(v[h][j + 2]),
+                            __uint_as_float(v[h][j + 3]));
+          __syncwarp();
+#pragma unroll
+          for (int rr = 0; rr < 32; rr += 4) {
+            const int t = quad * 32 + rr + sub_row;  // tile-local row
+            if (t < valid_rows && cc + col4 < p.E) {
+              const float4 val =
+                  *reinterpret_cast<const float4*>(my_scratch + (rr + sub_row) * PUSH_SCRATCH_STRIDE + col4);
+              float* dst = staging + static_cast<size_t>((t / C) * C + static_cast<int>(r)) * p.row_stride + cc + col4;
+              *reinterpret_cast<float4*>(__cluster_map_shared_rank(dst, static_cast<unsigned>(t % C))) = val;
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  cluster_arrive_release();  // every owner's staging area is complete past this point
+  cluster_wait_acquire();
+  if (warp == 1) {  // all tensor-memory reads of this CTA are done
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+
+  // ---------------- reduce owned rows, top-k, softmax ----------------
+  {
+    const int n_own = valid_rows > static_cast<int>(r) ? (valid_rows - static_cast<int>(r) + C - 1) / C : 0;
+    int group = 32;  // threads per owned row: a power of two
+    while (group > 1 && (n_own * group > SPLIT_THREADS || group * 8 > p.E)) group >>= 1;
+    const int rows_per_pass = SPLIT_THREADS / group;
+    const int passes = (n_own + rows_per_pass - 1) / rows_per_pass;
+    const int seg = threadIdx.x % group;
+    for (int pass = 0; pass < passes; ++pass) {
+      const int slot = pass * rows_per_pass + static_cast<int>(threadIdx.x) / group;
+      const bool active = slot < n_own;
+      RowTopK<KMAX> top;
+      top.reset();
+      if (active) {
+        // segment `seg` takes every group-th float4 of the row: consecutive lanes
+        // read consecutive 16-byte words (no bank conflicts), and each thread still
+        // offers its columns in increasing order
+        const float* rows = staging + static_cast<size_t>(slot) * C * p.row_stride;
+        const int c_end = p.E;
+        for (int c = 4 * seg; c < c_end; c += 4 * group) {
+          float4 v[C];
+#pragma unroll
+          for (int q = 0; q < C; ++q) v[q] = *reinterpret_cast<const float4*>(rows + q * p.row_stride + c);
+          float4 acc = v[0];
+#pragma unroll
+          for (int q = 1; q < C; ++q) {  // rank order: the same sum whichever CTA owns the row
+            acc.x += v[q].x;
+            acc.y += v[q].y;
+            acc.z += v[q].z;
+            acc.w += v[q].w;
+          }
+          top.offer(acc.x, c);
+          if (c + 1 < c_end) top.offer(acc.y, c + 1);
+          if (c + 2 < c_end) top.offer(acc.z, c + 2);
+          if (c + 3 < c_end) top.offer(acc.w, c + 3);
+        }
+      }
+      merge_lane_groups(top, group);
+      if (active && seg == 0) {
+        const int t_local = static_cast<int>(r) + C * slot;
+        const int64_t row = static_cast<int64_t>(tile) * BLOCK_M + t_local;
+        top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+      }
+    }
+  }
+
+}
+
+}  // namespace tkg

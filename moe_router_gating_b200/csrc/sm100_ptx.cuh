@@ -272,11 +272,15 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   return r;
 }
 
+// Every thread of the CTA calls these; the warp is reconverged first because the
+// barrier instruction is .aligned.
 __device__ __forceinline__ void cluster_arrive_release() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void cluster_wait_acquire() {
+  __syncwarp();
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 

@@ -10,6 +10,7 @@
 
 #include "tk_gating.h"
 #include "gating_row_tiles.cuh"
+#include "gating_split_h.cuh"
 
 namespace {
 
@@ -39,6 +40,35 @@ tk_status validate_sizes(int64_t T, int64_t H, int64_t E, int32_t k) {
   return TK_OK;
 }
 
+constexpr int kMaxSplit = 16;  // CTAs per cluster in the split-H variant (16 needs non-portable clusters)
+
+// Split-H plan: one 128-token tile per cluster of C CTAs, single-CTA MMAs.
+tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* plan) {
+  const int n_pad = round_up(static_cast<int>(E), 16);
+  const int b_boxes = (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+  const int stage_bytes = tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES;
+  const int scratch = tkg::PUSH_WARPS * tkg::PUSH_SCRATCH_BYTES;
+  int stages = (kMaxDynamicSmem - kSmemReserve - scratch) / stage_bytes;
+  if (stages > kMaxStages) stages = kMaxStages;
+  const int row_stride = round_up(static_cast<int>(E), 32) + 4;
+  // the staged partial rows of a tile reuse the ring
+  if (stages < 2 || tkg::BLOCK_M * row_stride * 4 > stages * stage_bytes) return TK_ERR_UNSUPPORTED;
+  const int64_t tiles = (T + tkg::BLOCK_M - 1) / tkg::BLOCK_M;
+  plan->variant = TK_VARIANT_SPLIT_H;
+  plan->block_m = tkg::BLOCK_M;
+  plan->n_pad = n_pad;
+  plan->num_tiles = static_cast<int32_t>(tiles);
+  plan->k_blocks = static_cast<int32_t>((H + tkg::BLOCK_K - 1) / tkg::BLOCK_K);
+  plan->split_h = C;
+  plan->stages = stages;
+  plan->grid = static_cast<int32_t>(tiles * C);
+  plan->cluster = C;
+  plan->threads = tkg::SPLIT_THREADS;
+  plan->smem_bytes = stages * stage_bytes + scratch + kSmemReserve;
+  plan->tmem_cols = static_cast<int32_t>(pow2_at_least(round_up(n_pad, 32)));
+  return TK_OK;
+}
+
 tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan) {
   if (plan == nullptr || num_sms < 1) return TK_ERR_INVALID_ARG;
   std::memset(plan, 0, sizeof(*plan));
@@ -47,6 +77,14 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   if (T == 0) {
     plan->variant = TK_VARIANT_NONE;
     return TK_OK;
+  }
+  const int64_t tiles128 = (T + tkg::BLOCK_M - 1) / tkg::BLOCK_M;
+  const int64_t k_blocks = (H + tkg::BLOCK_K - 1) / tkg::BLOCK_K;
+  if (tiles128 * 2 <= num_sms) {
+    // Few tiles: a cluster of C CTAs splits H for each 128-token tile.
+    int C = kMaxSplit;
+    while (C > 1 && (tiles128 * C > num_sms || C > k_blocks)) C >>= 1;
+    if (C >= 2) return plan_split_h(T, H, E, C, plan);
   }
   const bool pair = E > 64;  // gate halves of >= 64 experts per CTA (128-byte swizzle blocks)
   const int cg = pair ? 2 : 1;
@@ -108,30 +146,100 @@ bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-tk_status check_device(int* num_sms) {
+// Per-device facts and one-time kernel set-up, filled on the first call made with
+// that device current: compute capability, SM count, the device address of the
+// error word, every kernel's shared-memory limit (set to the maximum once, so no
+// per-call attribute calls), and the largest split-H cluster the device can
+// co-schedule.
+struct DeviceState {
+  bool ready = false;
+  tk_status status = TK_OK;
+  int num_sms = 0;
+  uint32_t* err_word = nullptr;
+  int max_split_cluster = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceState g_devices[kMaxDevices];
+std::mutex g_devices_mutex;
+
+template <typename Kernel>
+bool set_smem_limit(Kernel kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem) == cudaSuccess;
+}
+
+template <int KMAX>
+bool set_up_kernels() {
+  bool ok = set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 1>) &&
+            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2>) &&
+            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 2>) && set_smem_limit(tkg::gating_split_h_kernel<KMAX, 4>) &&
+            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 8>) && set_smem_limit(tkg::gating_split_h_kernel<KMAX, 16>);
+  return ok && cudaFuncSetAttribute(tkg::gating_split_h_kernel<KMAX, 16>,
+                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+}
+
+// Largest cluster size <= 16 (a power of two) of which at least one cluster of
+// full-shared-memory split-H CTAs fits on the device.
+int largest_schedulable_split_cluster() {
+  for (int C = 16; C >= 2; C >>= 1) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C);
+    cfg.blockDim = dim3(tkg::SPLIT_THREADS);
+    cfg.dynamicSmemBytes = kMaxDynamicSmem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    cudaError_t e = C == 16 ? cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 16>, &cfg)
+                            : cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 8>, &cfg);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    if (n > 0) return C;
+  }
+  return 0;
+}
+
+const DeviceState* device_state() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return TK_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState& d = g_devices[dev];
+  std::lock_guard<std::mutex> lock(g_devices_mutex);
+  if (d.ready) return &d;
   int major = 0, minor = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return TK_ERR_CUDA;
-  if (major != 10 || minor != 0) return TK_ERR_UNSUPPORTED;
-  return TK_OK;
-}
-
-uint32_t* device_error_word() {
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_tk_error_word) != cudaSuccess) return nullptr;
-  return static_cast<uint32_t*>(p);
+      cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (major != 10 || minor != 0) {
+    d.status = TK_ERR_UNSUPPORTED;
+    d.ready = true;
+    return &d;
+  }
+  void* err = nullptr;
+  if (cudaGetSymbolAddress(&err, g_tk_error_word) != cudaSuccess || !set_up_kernels<1>() || !set_up_kernels<2>() ||
+      !set_up_kernels<4>() || !set_up_kernels<8>() || !set_up_kernels<16>()) {
+    cudaGetLastError();
+    return nullptr;  // not cached: a later call retries
+  }
+  d.err_word = static_cast<uint32_t*>(err);
+  d.max_split_cluster = largest_schedulable_split_cluster();
+  d.status = TK_OK;
+  d.ready = true;
+  return &d;
 }
 
 template <int KMAX, int CG>
 tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mw,
                            const tkg::RowTileParams& prm, cudaStream_t stream) {
   auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem_bytes) != cudaSuccess)
-    return TK_ERR_CUDA;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
@@ -148,6 +256,40 @@ tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, cons
   return TK_OK;
 }
 
+template <int KMAX, int C>
+tk_status launch_split_h_c(const tk_gating_plan& plan, const CUtensorMap& mx, const CUtensorMap& mw,
+                           const tkg::SplitHParams& prm, cudaStream_t stream) {
+  auto kernel = tkg::gating_split_h_kernel<KMAX, C>;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.num_tiles * C);
+  cfg.blockDim = dim3(plan.threads);
+  cfg.dynamicSmemBytes = plan.smem_bytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, mx, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
+  return TK_OK;
+}
+
+template <int KMAX>
+tk_status launch_split_h(const tk_gating_plan& plan, int max_cluster, const CUtensorMap& mx, const CUtensorMap& mw,
+                         const tkg::SplitHParams& prm, cudaStream_t stream) {
+  int C = plan.cluster;
+  while (C > max_cluster) C >>= 1;  // the largest cluster the device co-schedules
+  switch (C) {
+    case 16: return launch_split_h_c<KMAX, 16>(plan, mx, mw, prm, stream);
+    case 8: return launch_split_h_c<KMAX, 8>(plan, mx, mw, prm, stream);
+    case 4: return launch_split_h_c<KMAX, 4>(plan, mx, mw, prm, stream);
+    case 2: return launch_split_h_c<KMAX, 2>(plan, mx, mw, prm, stream);
+    default: return TK_ERR_UNSUPPORTED;
+  }
+}
+
 template <int KMAX>
 tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mw,
                              const tkg::RowTileParams& prm, cudaStream_t stream) {
@@ -162,11 +304,11 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   if (T == 0) return TK_OK;
   if (!hidden || !gate || !scores || !ids) return TK_ERR_INVALID_ARG;
   if (!aligned16(hidden) || !aligned16(gate) || !aligned16(scores) || !aligned16(ids)) return TK_ERR_ALIGNMENT;
-  int num_sms = 0;
-  st = check_device(&num_sms);
-  if (st != TK_OK) return st;
+  const DeviceState* dev = device_state();
+  if (dev == nullptr) return TK_ERR_CUDA;
+  if (dev->status != TK_OK) return dev->status;
   tk_gating_plan pl;
-  st = plan_impl(T, H, E, k, num_sms, &pl);
+  st = plan_impl(T, H, E, k, dev->num_sms, &pl);
   if (st != TK_OK) return st;
 
   CUtensorMap mx, mw;
@@ -174,8 +316,31 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
                       tkg::BLOCK_M) ||
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
-  uint32_t* err = device_error_word();
-  if (err == nullptr) return TK_ERR_CUDA;
+  uint32_t* err = dev->err_word;
+
+  if (pl.variant == TK_VARIANT_SPLIT_H) {
+    tkg::SplitHParams sp;
+    sp.T = static_cast<int32_t>(T);
+    sp.H = static_cast<int32_t>(H);
+    sp.E = static_cast<int32_t>(E);
+    sp.k = k;
+    sp.n_pad = pl.n_pad;
+    sp.num_tiles = pl.num_tiles;
+    sp.k_blocks = pl.k_blocks;
+    sp.stages = pl.stages;
+    sp.b_boxes = (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+    sp.row_stride = round_up(static_cast<int>(E), 32) + 4;
+    sp.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
+    sp.timeout_ns = g_timeout_ns;
+    sp.scores = scores;
+    sp.ids = ids;
+    sp.err_word = err;
+    if (k <= 1) return launch_split_h<1>(pl, dev->max_split_cluster, mx, mw, sp, stream);
+    if (k <= 2) return launch_split_h<2>(pl, dev->max_split_cluster, mx, mw, sp, stream);
+    if (k <= 4) return launch_split_h<4>(pl, dev->max_split_cluster, mx, mw, sp, stream);
+    if (k <= 8) return launch_split_h<8>(pl, dev->max_split_cluster, mx, mw, sp, stream);
+    return launch_split_h<16>(pl, dev->max_split_cluster, mx, mw, sp, stream);
+  }
 
   tkg::RowTileParams prm;
   prm.T = static_cast<int32_t>(T);

@@ -89,10 +89,30 @@ def test_plans_for_router_workloads():
         if p["variant"] == 3:
             assert p["cluster"] == 2 and p["block_m"] == 256 and p["n_pad"] in (128, 256)
             assert p["grid"] == 2 * min(p["num_tiles"], 74)
+        if p["variant"] == 2:
+            C = p["cluster"]
+            assert C in (2, 4, 8, 16) and p["split_h"] == C and C <= p["k_blocks"]
+            assert p["grid"] == p["num_tiles"] * C <= 148
+
+
+def test_plan_variant_choice():
+    # few tiles: split H across a cluster; many tiles: persistent row tiles / pairs
+    assert tk.make_plan(1, 7168, 256, 8)["variant"] == 2
+    assert tk.make_plan(1, 7168, 256, 8)["cluster"] == 16
+    assert tk.make_plan(4096, 7168, 256, 8)["cluster"] == 4
+    assert tk.make_plan(8192, 7168, 256, 8)["cluster"] == 2
+    assert tk.make_plan(65536, 7168, 256, 8)["variant"] == 3
+    assert tk.make_plan(16384, 4096, 64, 6)["variant"] == 1
+    assert tk.make_plan(130, 8, 256, 8)["variant"] == 3      # one k-block: nothing to split
+    p = tk.make_plan(300, 520, 40, 3)                        # 9 k-blocks: cluster capped at 8
+    assert p["variant"] == 2 and p["cluster"] == 8
 
 
 def test_plan_tmem_and_smem_budget():
-    for E in range(16, 257, 8):
-        p = tk.make_plan(1000, 7168, E, min(8, E), 148)
-        assert p["tmem_cols"] >= 2 * ((p["n_pad"] + 31) // 32 * 32)
-        assert p["smem_bytes"] <= 232448
+    for T in (1, 1000, 30000):
+        for E in range(16, 257, 8):
+            p = tk.make_plan(T, 7168, E, min(8, E), 148)
+            buffers = 1 if p["variant"] == 2 else 2  # split-H keeps one accumulator
+            assert p["tmem_cols"] >= buffers * ((p["n_pad"] + 31) // 32 * 32)
+            assert p["tmem_cols"] <= 512
+            assert p["smem_bytes"] <= 232448
