@@ -120,7 +120,7 @@ typedef struct {
   int32_t variant;      /* tk_variant */
   int32_t block_m;      /* tokens per tile */
   int32_t n_pad;        /* MMA N: E rounded up to a multiple of 16 */
-  int32_t num_tiles;    /* ceil(T / block_m) */
+  int32_t num_tiles;    /* full tiles of block_m tokens (all of T unless num_half_tiles > 0) */
   int32_t k_blocks;     /* ceil(H / 64) */
   int32_t split_h;      /* CTAs sharing one tile's H range (1 = none) */
   int32_t stages;       /* shared-memory ring depth */
@@ -129,12 +129,16 @@ typedef struct {
   int32_t threads;      /* threads per CTA */
   int32_t smem_bytes;   /* dynamic shared memory per CTA */
   int32_t tmem_cols;    /* tensor-memory columns allocated per CTA */
+  int32_t num_half_tiles; /* CTA pairs: 128-token tiles after the full ones (balanced last round) */
 } tk_gating_plan;
 
 /*
  * tk_gating_make_plan -- fill *plan with the launch tk_gating_fused_topk makes
- * for (T, H, E, k) on a device with `num_sms` SMs.  Validates like
- * tk_gating_fused_topk (pointers excepted).  Makes no CUDA call.
+ * for (T, H, E, k) on a device with `num_sms` SMs whose clusters fit like a
+ * B200's (of 148 SMs, 74 / 33 / 15 / 7 clusters of 2 / 4 / 8 / 16 CTAs run at
+ * once; scaled by num_sms / 148).  The launch itself uses the current device's
+ * measured cluster capacities, so on other parts the cluster size may differ.
+ * Validates like tk_gating_fused_topk (pointers excepted).  Makes no CUDA call.
  */
 TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan);
 

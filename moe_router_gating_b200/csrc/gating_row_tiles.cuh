@@ -11,6 +11,11 @@
 //   both CTAs' shared memory and write each CTA's 128 rows x N logits into its
 //   own tensor memory.  Per CTA this halves the gate bytes each tile pulls from
 //   L2 compared with CG = 1.
+//   Balanced tail: when the last round of 256-token tiles would leave pairs
+//   idle, the remaining rows run as 128-token "half" tiles (M = 128 pair MMAs,
+//   64 rows per CTA), which take half the MMA time of a full tile.  A half-tile
+//   accumulator is folded in tensor memory: lanes 0..63 hold the CTA's 64 rows
+//   for experts [0, N/2) and lanes 64..127 the same rows for experts [N/2, N).
 //
 // Warp roles (192 threads per CTA):
 //   warp 0      TMA producer: 64-wide K slices of the hidden rows (K-major,
@@ -30,6 +35,7 @@
 
 #include "sm100_ptx.cuh"
 #include "topk_epilogue.cuh"
+#include "topk_merge.cuh"
 
 namespace tkg {
 
@@ -46,7 +52,8 @@ struct RowTileParams {
   int32_t T, H, E, k;
   int32_t n_pad;        // MMA N (CG=1: E rounded up to 16; CG=2: 128 or 256)
   int32_t acc_stride;   // TMEM columns between the two accumulator buffers
-  int32_t num_tiles;    // tiles of BLOCK_M * CG rows
+  int32_t num_tiles;    // full tiles of BLOCK_M * CG rows, starting at row 0
+  int32_t num_half;     // pairs only: half tiles of BLOCK_M rows after the full tiles
   int32_t k_blocks;
   int32_t stages;
   int32_t b_boxes;      // gate boxes per stage loaded by each CTA
@@ -73,24 +80,49 @@ __device__ __forceinline__ uint64_t b_desc_k_slice(uint32_t b_stage_addr, int kk
   return smem_desc_sw128(b_stage_addr + kk * (UMMA_K / 8) * 1024, B_BOX_BYTES, 1024);
 }
 
-// Offer 32 consecutive logits (columns c0 .. c0+31) of this thread's row;
-// columns at or beyond E (MMA padding) are skipped.
+// The i-th tile of a CTA (or pair) `unit` out of `units`: full tiles round-robin,
+// then at most one half tile.  Returns false past the end of its list.
+struct TileWork {
+  int row0;   // first token row of the tile (pair tile: of the pair)
+  bool half;  // 128-token pair tile
+};
+
+template <int CG>
+__device__ __forceinline__ bool tile_work(const RowTileParams& p, int unit, int units, int i, TileWork& w) {
+  const int n_full = unit < p.num_tiles ? (p.num_tiles - 1 - unit) / units + 1 : 0;
+  if (i < n_full) {
+    w.row0 = (unit + i * units) * (BLOCK_M * CG);
+    w.half = false;
+    return true;
+  }
+  if (CG == 2 && i == n_full && unit < p.num_half) {
+    w.row0 = p.num_tiles * (BLOCK_M * CG) + unit * BLOCK_M;
+    w.half = true;
+    return true;
+  }
+  return false;
+}
+
+// Offer 32 consecutive logits (accumulator columns c0 .. c0+31, expert ids
+// col_base + c0 ..) of this thread's row; columns at or beyond ncols (MMA
+// padding) are skipped.
 template <int KMAX>
-__device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (&r)[32], int c0, int E) {
-  if (c0 + 32 <= E) {
+__device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (&r)[32], int c0, int ncols,
+                                            int col_base) {
+  if (c0 + 32 <= ncols) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) top.offer(__uint_as_float(r[j]), c0 + j);
+    for (int j = 0; j < 32; ++j) top.offer(__uint_as_float(r[j]), col_base + c0 + j);
   } else {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (c0 + j < E) top.offer(__uint_as_float(r[j]), c0 + j);
+      if (c0 + j < ncols) top.offer(__uint_as_float(r[j]), col_base + c0 + j);
   }
 }
 
 template <int KMAX, int CG>
 __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
-    gating_row_tiles_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
-                            const RowTileParams p) {
+    gating_row_tiles_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_x64,
+                            const __grid_constant__ CUtensorMap map_w, const RowTileParams p) {
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
   constexpr bool kPair = CG == 2;
   extern __shared__ uint8_t smem_dyn[];
@@ -109,8 +141,8 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = kPair ? cluster_ctarank() : 0;  // 0 = the pair's MMA leader
   const bool leader = rank == 0;
-  const int first_tile = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int tile_step = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -125,6 +157,7 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&map_x);
+    if (kPair && p.num_half > 0) tma_prefetch_desc(&map_x64);
     tma_prefetch_desc(&map_w);
   }
   if (warp == 1) {
@@ -152,13 +185,16 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       // ---------------- TMA producer ----------------
       const uint64_t pol_x = l2_policy_evict_first();  // hidden: streamed once
       const uint64_t pol_w = l2_policy_evict_last();   // gate: re-read by every tile
-      const uint32_t stage_tx = CG * (A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES);
       const int b_col0 = static_cast<int>(rank) * p.b_boxes * B_BOX_N;  // this CTA's gate columns
       uint32_t stage = 0, phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int tile = first_tile; ok && tile < p.num_tiles; tile += tile_step) {
-        const int row0 = tile * (BLOCK_M * CG) + static_cast<int>(rank) * BLOCK_M;
+      TileWork w;
+      for (int item = 0; ok && tile_work<CG>(p, unit, units, item, w); ++item) {
+        const int cta_rows = w.half ? BLOCK_M / 2 : BLOCK_M;  // hidden rows this CTA stages
+        const int row0 = w.row0 + static_cast<int>(rank) * cta_rows;
+        const uint32_t stage_tx = CG * (cta_rows * BLOCK_K * 2 + p.b_boxes * B_BOX_BYTES);
+        const CUtensorMap* map_a = w.half ? &map_x64 : &map_x;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER, p.err_word)) {
             ok = false;
@@ -167,7 +203,7 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
           if constexpr (kPair) {
             const uint32_t bar = map_shared_rank(smem_u32(&full[stage]), 0);
-            tma_load_2d_pair(sA + stage * A_STAGE_BYTES, &map_x, bar, kb * BLOCK_K, row0, pol_x);
+            tma_load_2d_pair(sA + stage * A_STAGE_BYTES, map_a, bar, kb * BLOCK_K, row0, pol_x);
             for (int j = 0; j < p.b_boxes; ++j)
               tma_load_2d_pair(sB + (stage * p.b_boxes + j) * B_BOX_BYTES, &map_w, bar, b_col0 + j * B_BOX_N,
                                kb * BLOCK_K, pol_w);
@@ -196,20 +232,23 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           } else {
             --stage;
           }
-          mbar_wait(&full[stage], phase, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
+          mbar_wait(&full[stage], phase, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer ----------------
-      const uint32_t idesc = idesc_bf16_f32(BLOCK_M * CG, p.n_pad, false, true);
+      const uint32_t idesc_full = idesc_bf16_f32(BLOCK_M * CG, p.n_pad, false, true);
+      const uint32_t idesc_half = idesc_bf16_f32(BLOCK_M, p.n_pad, false, true);  // pairs: 64 rows per CTA
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
-      for (int tile = first_tile; ok && tile < p.num_tiles; tile += tile_step, ++local) {
+      TileWork w;
+      for (; ok && tile_work<CG>(p, unit, units, local, w); ++local) {
         const uint32_t buf = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
+        const uint32_t idesc = w.half ? idesc_half : idesc_full;
         if (!mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + buf * p.acc_stride;
@@ -250,7 +289,7 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
         umma_commit_pair(drain);
       else
         umma_commit(drain);
-      mbar_wait(drain, 0, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
+      mbar_wait(drain, 0, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
     }
     __syncwarp();
   } else {
@@ -258,25 +297,31 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     const int quad = warp & 3;  // TMEM lanes this warp may access
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int local = 0;
-    for (int tile = first_tile; tile < p.num_tiles; tile += tile_step, ++local) {
+    TileWork w;
+    for (; tile_work<CG>(p, unit, units, local, w); ++local) {
       const uint32_t buf = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       bool ok = mbar_wait(&acc_full[buf], acc_phase, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
 
+      // full tile: one row per thread over all experts; half tile: lanes 0..63
+      // hold experts [0, N/2) and lanes 64..127 experts [N/2, N) of 64 rows
+      const bool upper = w.half && quad >= 2;
+      const int col_base = upper ? p.n_pad / 2 : 0;
+      const int ncols = w.half ? min(p.n_pad / 2, p.E - col_base) : p.E;
       RowTopK<KMAX> top;
       top.reset();
       const uint32_t acc_addr = lane_base + buf * p.acc_stride;
       // 64 columns per round trip: two loads, one wait
-      for (int c0 = 0; c0 < p.E; c0 += 64) {
+      for (int c0 = 0; c0 < ncols; c0 += 64) {
         uint32_t r0[32], r1[32];
-        const bool second = c0 + 32 < p.E;  // warp-uniform
+        const bool second = c0 + 32 < ncols;  // warp-uniform
         tmem_ld_32(acc_addr + c0, r0);
         if (second) tmem_ld_32(acc_addr + c0 + 32, r1);
         tmem_ld_wait();
-        offer_chunk(top, r0, c0, p.E);
-        if (second) offer_chunk(top, r1, c0 + 32, p.E);
+        offer_chunk(top, r0, c0, ncols, col_base);
+        if (second) offer_chunk(top, r1, c0 + 32, ncols, col_base);
       }
       // the accumulator buffer may be overwritten once every epilogue warp of
       // the pair has read it
@@ -289,13 +334,42 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           mbar_arrive(&acc_empty[buf]);
       }
 
-      const int64_t row = static_cast<int64_t>(tile) * (BLOCK_M * CG) + rank * BLOCK_M + quad * 32 + lane;
-      if (row < p.T) top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+      if (!w.half) {
+        const int64_t row = static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
+        if (row < p.T) top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+      } else {
+        // A half tile is a CTA's last tile, so its ring is idle: the upper lanes
+        // hand their lists to the lower lanes of the same rows through it.
+        const int m = (quad & 1) * 32 + lane;  // row within this CTA's 64
+        float* xv = reinterpret_cast<float*>(sA) + m * KMAX;
+        int32_t* xi = reinterpret_cast<int32_t*>(sA + BLOCK_M * KMAX * 4) + m * KMAX;
+        if (upper) {
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) {
+            xv[j] = top.v[j];
+            xi[j] = top.i[j];
+          }
+        }
+        named_barrier_sync(1, NUM_EPI_WARPS * 32);
+        if (!upper) {
+          float bv[KMAX];
+          int32_t bi[KMAX];
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) {
+            bv[j] = xv[j];
+            bi[j] = xi[j];
+          }
+          merge_sorted(top, bv, bi);
+          const int64_t row = static_cast<int64_t>(w.row0) + rank * (BLOCK_M / 2) + m;
+          if (row < p.T) top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+        }
+      }
     }
   }
 
   tc_fence_before_sync();
   if constexpr (kPair) {
+    settle_after_abort(abort_flag);
     // neither CTA frees its shared or tensor memory while the pair still uses it
     cluster_arrive_release();
     cluster_wait_acquire();

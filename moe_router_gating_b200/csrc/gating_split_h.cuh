@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
         } else {
           --stage;
         }
-        mbar_wait(&full[stage], phase, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
+        mbar_wait(&full[stage], phase, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
       }
     }
   } else if (warp == 1) {
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
       }
       if (ok) umma_commit(acc_full);
       umma_commit(drain);
-      mbar_wait(drain, 0, nullptr, p.timeout_ns, ERR_WAIT_DRAIN, p.err_word);
+      mbar_wait(drain, 0, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
     }
     __syncwarp();
   }

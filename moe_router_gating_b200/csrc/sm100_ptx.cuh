@@ -11,6 +11,16 @@
 
 namespace tkg {
 
+// Limit of the waits that let a stopping kernel's own copies and MMAs finish
+// (drains): independent of the configurable wait limit, so an early abort never
+// leaves an asynchronous copy in flight when the CTA exits.
+constexpr uint64_t DRAIN_TIMEOUT_NS = 1000000000ull;
+// After an abort, a CTA of a pair also pauses this long before leaving: the
+// peer's loads complete on the leader's barriers, which the peer cannot wait on.
+constexpr uint64_t ABORT_SETTLE_NS = 100000ull;
+
+__device__ __forceinline__ void settle_after_abort(volatile int* abort_flag);
+
 // ---- device error word (read by the host entry point tk_gating_device_error) ----
 enum : uint32_t {
   ERR_WAIT_PRODUCER = 1u << 0,
@@ -66,20 +76,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that suspends the thread for at most `suspend_ns` before reporting
+// that the phase is still incomplete.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Polling granularity of the bounded waits.
+constexpr uint32_t WAIT_POLL_NS = 20000;
+
 // Waits until the phase with the given parity has completed.  Returns false on
-// timeout or when *abort is set; on timeout it sets *abort and ORs `code` into
-// the device error word.
+// timeout (checked every WAIT_POLL_NS at most) or when *abort is set; on timeout
+// it sets *abort and ORs `code` into the device error word.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns, uint32_t code, uint32_t* err_word) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_for(bar, parity, WAIT_POLL_NS)) return true;
     if (abort != nullptr && *abort) return false;
     if (globaltimer_ns() - t0 > timeout_ns) {
       if (abort != nullptr) *abort = 1;
       atomicOr(err_word, code);
       return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void settle_after_abort(volatile int* abort_flag) {
+  if (abort_flag != nullptr && *abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < ABORT_SETTLE_NS) {
     }
   }
 }
@@ -289,6 +324,11 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t smem_addr, uint32_t
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
   return r;
+}
+
+// Named barrier among `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Arrive on an mbarrier of another CTA of the cluster (address from mapa).

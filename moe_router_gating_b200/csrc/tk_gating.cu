@@ -69,7 +69,32 @@ tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* p
   return TK_OK;
 }
 
-tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan) {
+// Clusters of 2^i CTAs (one CTA per SM) that a device runs at once, i = 0..4.
+// Measured on B200 (148 SMs): 148, 74, 33, 15, 7 -- GPCs do not divide evenly
+// into 4-, 8- and 16-SM groups.  Scaled for other SM counts when planning
+// without a device; launches use the device's own figures.
+struct ClusterCapacity {
+  int n[5];
+};
+
+ClusterCapacity b200_like_capacity(int num_sms) {
+  ClusterCapacity c;
+  c.n[0] = num_sms;
+  c.n[1] = num_sms / 2;
+  c.n[2] = num_sms * 33 / 148;
+  c.n[3] = num_sms * 15 / 148;
+  c.n[4] = num_sms * 7 / 148;
+  return c;
+}
+
+int log2_of(int c) {
+  int i = 0;
+  while ((1 << i) < c) ++i;
+  return i;
+}
+
+tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, const ClusterCapacity& cap,
+                    tk_gating_plan* plan) {
   if (plan == nullptr || num_sms < 1) return TK_ERR_INVALID_ARG;
   std::memset(plan, 0, sizeof(*plan));
   tk_status st = validate_sizes(T, H, E, k);
@@ -81,9 +106,10 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   const int64_t tiles128 = (T + tkg::BLOCK_M - 1) / tkg::BLOCK_M;
   const int64_t k_blocks = (H + tkg::BLOCK_K - 1) / tkg::BLOCK_K;
   if (tiles128 * 2 <= num_sms) {
-    // Few tiles: a cluster of C CTAs splits H for each 128-token tile.
+    // Few tiles: a cluster of C CTAs splits H for each 128-token tile; C is the
+    // largest size whose clusters all run at once (one wave).
     int C = kMaxSplit;
-    while (C > 1 && (tiles128 * C > num_sms || C > k_blocks)) C >>= 1;
+    while (C > 1 && (tiles128 > cap.n[log2_of(C)] || C > k_blocks)) C >>= 1;
     if (C >= 2) return plan_split_h(T, H, E, C, plan);
   }
   const bool pair = E > 64;  // gate halves of >= 64 experts per CTA (128-byte swizzle blocks)
@@ -96,8 +122,22 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return TK_ERR_UNSUPPORTED;
   const int64_t rows_per_tile = static_cast<int64_t>(tkg::BLOCK_M) * cg;
-  const int64_t tiles = (T + rows_per_tile - 1) / rows_per_tile;
-  const int64_t units = num_sms / cg;  // CTAs (or CTA pairs) resident at once
+  int64_t tiles = (T + rows_per_tile - 1) / rows_per_tile;
+  const int64_t units_max = num_sms / cg;  // CTAs (or CTA pairs) resident at once
+  const int64_t units = tiles < units_max ? tiles : units_max;
+  int64_t half_tiles = 0;
+  if (pair) {
+    // Balanced tail: count work in 128-row units (a full pair tile is 2).  After
+    // F full rounds, if the u units left fit one per pair, run them as half tiles
+    // (half the MMA time) instead of a partly idle round of full tiles.
+    const int64_t h = (T + tkg::BLOCK_M - 1) / tkg::BLOCK_M;
+    const int64_t F = h / (2 * units);
+    const int64_t u = h - 2 * units * F;
+    if (F >= 1 && u > 0 && u <= units) {
+      tiles = F * units;
+      half_tiles = u;
+    }
+  }
 
   plan->variant = pair ? TK_VARIANT_ROW_PAIRS : TK_VARIANT_ROW_TILES;
   plan->block_m = static_cast<int32_t>(rows_per_tile);
@@ -106,7 +146,8 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   plan->k_blocks = static_cast<int32_t>((H + tkg::BLOCK_K - 1) / tkg::BLOCK_K);
   plan->split_h = 1;
   plan->stages = stages;
-  plan->grid = static_cast<int32_t>((tiles < units ? tiles : units) * cg);
+  plan->grid = static_cast<int32_t>(units * cg);
+  plan->num_half_tiles = static_cast<int32_t>(half_tiles);
   plan->cluster = cg;
   plan->threads = tkg::ROW_TILE_THREADS;
   plan->smem_bytes = stages * stage_bytes + kSmemReserve;
@@ -157,6 +198,7 @@ struct DeviceState {
   int num_sms = 0;
   uint32_t* err_word = nullptr;
   int max_split_cluster = 0;
+  ClusterCapacity capacity = {};
 };
 
 constexpr int kMaxDevices = 64;
@@ -178,10 +220,13 @@ bool set_up_kernels() {
                                     cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
 }
 
-// Largest cluster size <= 16 (a power of two) of which at least one cluster of
-// full-shared-memory split-H CTAs fits on the device.
-int largest_schedulable_split_cluster() {
-  for (int C = 16; C >= 2; C >>= 1) {
+// Clusters of each size 2^i (i = 1..4) of full-shared-memory CTAs that the
+// device runs at once.
+ClusterCapacity measure_cluster_capacity(int num_sms) {
+  ClusterCapacity cap;
+  cap.n[0] = num_sms;
+  for (int i = 1; i <= 4; ++i) {
+    const int C = 1 << i;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = C;
@@ -200,9 +245,9 @@ int largest_schedulable_split_cluster() {
       cudaGetLastError();
       n = 0;
     }
-    if (n > 0) return C;
+    cap.n[i] = n;
   }
-  return 0;
+  return cap;
 }
 
 const DeviceState* device_state() {
@@ -230,15 +275,21 @@ const DeviceState* device_state() {
     return nullptr;  // not cached: a later call retries
   }
   d.err_word = static_cast<uint32_t*>(err);
-  d.max_split_cluster = largest_schedulable_split_cluster();
+  d.capacity = measure_cluster_capacity(d.num_sms);
+  d.max_split_cluster = 0;
+  for (int i = 4; i >= 1; --i)
+    if (d.capacity.n[i] > 0) {
+      d.max_split_cluster = 1 << i;
+      break;
+    }
   d.status = TK_OK;
   d.ready = true;
   return &d;
 }
 
 template <int KMAX, int CG>
-tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mw,
-                           const tkg::RowTileParams& prm, cudaStream_t stream) {
+tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
+                           const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
   auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -252,7 +303,7 @@ tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, cons
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = CG > 1 ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, kernel, mx, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kernel, mx, mx64, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
   return TK_OK;
 }
 
@@ -291,10 +342,10 @@ tk_status launch_split_h(const tk_gating_plan& plan, int max_cluster, const CUte
 }
 
 template <int KMAX>
-tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mw,
-                             const tkg::RowTileParams& prm, cudaStream_t stream) {
-  if (pl.variant == TK_VARIANT_ROW_PAIRS) return launch_row_tiles<KMAX, 2>(pl, mx, mw, prm, stream);
-  return launch_row_tiles<KMAX, 1>(pl, mx, mw, prm, stream);
+tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
+                             const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
+  if (pl.variant == TK_VARIANT_ROW_PAIRS) return launch_row_tiles<KMAX, 2>(pl, mx, mx64, mw, prm, stream);
+  return launch_row_tiles<KMAX, 1>(pl, mx, mx64, mw, prm, stream);
 }
 
 tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int64_t H, int64_t E, int32_t k,
@@ -308,12 +359,15 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   if (dev == nullptr) return TK_ERR_CUDA;
   if (dev->status != TK_OK) return dev->status;
   tk_gating_plan pl;
-  st = plan_impl(T, H, E, k, dev->num_sms, &pl);
+  st = plan_impl(T, H, E, k, dev->num_sms, dev->capacity, &pl);
   if (st != TK_OK) return st;
 
-  CUtensorMap mx, mw;
+  CUtensorMap mx, mx64, mw;
+  std::memset(&mx64, 0, sizeof(mx64));
   if (!encode_2d_bf16(&mx, hidden, static_cast<uint64_t>(T), static_cast<uint64_t>(H), tkg::BLOCK_K,
                       tkg::BLOCK_M) ||
+      (pl.num_half_tiles > 0 && !encode_2d_bf16(&mx64, hidden, static_cast<uint64_t>(T), static_cast<uint64_t>(H),
+                                                tkg::BLOCK_K, tkg::BLOCK_M / 2)) ||
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
   uint32_t* err = dev->err_word;
@@ -350,6 +404,7 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   prm.n_pad = pl.n_pad;
   prm.acc_stride = round_up(pl.n_pad, 32);
   prm.num_tiles = pl.num_tiles;
+  prm.num_half = pl.num_half_tiles;
   prm.k_blocks = pl.k_blocks;
   prm.stages = pl.stages;
   prm.b_boxes = pl.variant == TK_VARIANT_ROW_PAIRS ? pl.n_pad / 2 / tkg::B_BOX_N
@@ -360,11 +415,11 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   prm.ids = ids;
   prm.err_word = err;
 
-  if (k <= 1) return launch_row_variant<1>(pl, mx, mw, prm, stream);
-  if (k <= 2) return launch_row_variant<2>(pl, mx, mw, prm, stream);
-  if (k <= 4) return launch_row_variant<4>(pl, mx, mw, prm, stream);
-  if (k <= 8) return launch_row_variant<8>(pl, mx, mw, prm, stream);
-  return launch_row_variant<16>(pl, mx, mw, prm, stream);
+  if (k <= 1) return launch_row_variant<1>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 2) return launch_row_variant<2>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 4) return launch_row_variant<4>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 8) return launch_row_variant<8>(pl, mx, mx64, mw, prm, stream);
+  return launch_row_variant<16>(pl, mx, mx64, mw, prm, stream);
 }
 
 }  // namespace
@@ -400,7 +455,8 @@ tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* gate_we
 }
 
 tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan) {
-  return plan_impl(T, H, E, k, num_sms, plan);
+  if (num_sms < 1) return TK_ERR_INVALID_ARG;
+  return plan_impl(T, H, E, k, num_sms, b200_like_capacity(num_sms), plan);
 }
 
 tk_status tk_gating_device_error(uint32_t* word, int32_t clear) {

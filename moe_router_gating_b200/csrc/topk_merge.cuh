@@ -20,20 +20,14 @@ __device__ __forceinline__ bool ranks_before(float va, int32_t ia, float vb, int
   return va > vb || (va == vb && ia < ib);
 }
 
+// t <- the best L entries of t U (bv, bi), sorted; (bv, bi) is a sorted list of L.
 template <int L>
-__device__ __forceinline__ void merge_with_lane(RowTopK<L>& t, int lane_mask) {
-  float pv[L];
-  int32_t pi[L];
+__device__ __forceinline__ void merge_sorted(RowTopK<L>& t, const float (&bv)[L], const int32_t (&bi)[L]) {
 #pragma unroll
   for (int j = 0; j < L; ++j) {
-    pv[j] = __shfl_xor_sync(0xffffffffu, t.v[j], lane_mask);
-    pi[j] = __shfl_xor_sync(0xffffffffu, t.i[j], lane_mask);
-  }
-#pragma unroll
-  for (int j = 0; j < L; ++j) {
-    const bool take = ranks_before(pv[L - 1 - j], pi[L - 1 - j], t.v[j], t.i[j]);
-    t.v[j] = take ? pv[L - 1 - j] : t.v[j];
-    t.i[j] = take ? pi[L - 1 - j] : t.i[j];
+    const bool take = ranks_before(bv[L - 1 - j], bi[L - 1 - j], t.v[j], t.i[j]);
+    t.v[j] = take ? bv[L - 1 - j] : t.v[j];
+    t.i[j] = take ? bi[L - 1 - j] : t.i[j];
   }
 #pragma unroll
   for (int d = L / 2; d >= 1; d /= 2) {
@@ -50,6 +44,18 @@ __device__ __forceinline__ void merge_with_lane(RowTopK<L>& t, int lane_mask) {
       }
     }
   }
+}
+
+template <int L>
+__device__ __forceinline__ void merge_with_lane(RowTopK<L>& t, int lane_mask) {
+  float pv[L];
+  int32_t pi[L];
+#pragma unroll
+  for (int j = 0; j < L; ++j) {
+    pv[j] = __shfl_xor_sync(0xffffffffu, t.v[j], lane_mask);
+    pi[j] = __shfl_xor_sync(0xffffffffu, t.i[j], lane_mask);
+  }
+  merge_sorted(t, pv, pi);
 }
 
 // Merge the lists of groups of `group` consecutive lanes (a power of two <= 32).

@@ -95,6 +95,19 @@ def test_plans_for_router_workloads():
             assert p["grid"] == p["num_tiles"] * C <= 148
 
 
+def test_plan_half_tiles_cover_rows_once():
+    for T in (9473, 18945, 19999, 20000, 30000, 60000, 65536, 100000):
+        p = tk.make_plan(T, 512, 256, 8, 148)
+        if p["variant"] != 3:
+            continue
+        pairs = p["grid"] // 2
+        rows = p["num_tiles"] * 256 + p["num_half_tiles"] * 128
+        assert rows >= T and rows - T < 256
+        assert p["num_half_tiles"] <= pairs
+        if p["num_half_tiles"]:
+            assert p["num_tiles"] % pairs == 0  # every pair: the same full tiles, then one half tile
+
+
 def test_plan_variant_choice():
     # few tiles: split H across a cluster; many tiles: persistent row tiles / pairs
     assert tk.make_plan(1, 7168, 256, 8)["variant"] == 2

@@ -83,6 +83,8 @@ def test_train_workload_sampled_rows():
     (1, 64, 16, 1), (127, 64, 16, 16), (129, 72, 24, 5), (300, 520, 40, 3), (1000, 256, 64, 8),
     (257, 128, 200, 7), (640, 1024, 256, 16), (130, 8, 256, 8), (2500, 96, 136, 4), (5000, 512, 256, 2),
     (20000, 256, 256, 8), (19000, 128, 40, 3), (10000, 7168, 256, 8), (100, 7168, 256, 16), (3, 2048, 64, 4),
+    # CTA pairs with a balanced last round of 128-token tiles (E padding in the upper expert half)
+    (19999, 512, 200, 8), (60000, 512, 136, 16), (18945, 1024, 256, 1),
 ])
 def test_ragged_shapes(T, H, E, k):
     wl = workloads.RouterWorkload(f"shape_{T}_{H}_{E}_{k}", T, H, E, k, seed=3)
