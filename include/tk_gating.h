@@ -123,7 +123,7 @@ typedef struct {
   int32_t num_tiles;    /* full tiles of block_m tokens (all of T unless num_half_tiles > 0) */
   int32_t k_blocks;     /* ceil(H / 64) */
   int32_t split_h;      /* CTAs sharing one tile's H range (1 = none) */
-  int32_t stages;       /* shared-memory ring depth */
+  int32_t stages;       /* shared-memory ring depth (row tiles: stages of two 64-wide K slices) */
   int32_t grid;         /* CTAs launched */
   int32_t cluster;      /* CTAs per cluster */
   int32_t threads;      /* threads per CTA */

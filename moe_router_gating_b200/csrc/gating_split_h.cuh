@@ -63,9 +63,9 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align_1024(smem_dyn);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + p.stages * A_STAGE_BYTES;
+  uint8_t* sB = smem + p.stages * KB_PER_STAGE * A_STAGE_BYTES;
   float* staging = reinterpret_cast<float*>(smem);  // reuses the ring once every CTA's MMAs are done
-  float* scratch = reinterpret_cast<float*>(sB + p.stages * p.b_boxes * B_BOX_BYTES);  // after the ring
+  float* scratch = reinterpret_cast<float*>(sB + p.stages * KB_PER_STAGE * p.b_boxes * B_BOX_BYTES);  // after the ring
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scratch) + PUSH_WARPS * PUSH_SCRATCH_BYTES);
   uint64_t* empty = full + p.stages;
   uint64_t* acc_full = empty + p.stages;
@@ -108,16 +108,21 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
       // ---------------- TMA producer: this CTA's H slice of one tile ----------------
       const uint64_t pol_x = l2_policy_evict_first();
       const uint64_t pol_w = l2_policy_evict_last();
-      const uint32_t stage_tx = A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES;
+      const uint32_t slice_tx = A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES;
       uint32_t stage = 0, phase = 0;
       int issued = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1; kb += KB_PER_STAGE) {
+        // a stage holds up to KB_PER_STAGE slices, never past this CTA's H slice
+        const int n_sub = min(KB_PER_STAGE, kb1 - kb);
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER, p.err_word)) break;
-        mbar_arrive_expect_tx(&full[stage], stage_tx);
-        tma_load_2d(sA + stage * A_STAGE_BYTES, &map_x, &full[stage], kb * BLOCK_K, tile * BLOCK_M, pol_x);
-        for (int j = 0; j < p.b_boxes; ++j)
-          tma_load_2d(sB + (stage * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], j * B_BOX_N, kb * BLOCK_K,
-                      pol_w);
+        mbar_arrive_expect_tx(&full[stage], n_sub * slice_tx);
+        for (int sub = 0; sub < n_sub; ++sub) {
+          const int slot = stage * KB_PER_STAGE + sub;
+          const int k0 = (kb + sub) * BLOCK_K;
+          tma_load_2d(sA + slot * A_STAGE_BYTES, &map_x, &full[stage], k0, tile * BLOCK_M, pol_x);
+          for (int j = 0; j < p.b_boxes; ++j)
+            tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], j * B_BOX_N, k0, pol_w);
+        }
         ++issued;
         if (++stage == static_cast<uint32_t>(p.stages)) {
           stage = 0;
@@ -141,17 +146,22 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
       const uint32_t idesc = idesc_bf16_f32(BLOCK_M, p.n_pad, false, true);
       uint32_t stage = 0, phase = 0;
       bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1; kb += KB_PER_STAGE) {
+        const int n_sub = min(KB_PER_STAGE, kb1 - kb);
         if (!mbar_wait(&full[stage], phase, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
-        const uint32_t b_addr = smem_u32(sB + stage * p.b_boxes * B_BOX_BYTES);
+        for (int sub = 0; sub < n_sub; ++sub) {
+          const int slot = stage * KB_PER_STAGE + sub;
+          const uint32_t a_addr = smem_u32(sA + slot * A_STAGE_BYTES);
+          const uint32_t b_addr = smem_u32(sB + slot * p.b_boxes * B_BOX_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
-          umma_bf16(tmem_base, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc, (kb != kb0) | kk);
+          for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
+            umma_bf16(tmem_base, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc,
+                      (kb + sub != kb0) | kk);
+        }
         umma_commit(&empty[stage]);
         if (++stage == static_cast<uint32_t>(p.stages)) {
           stage = 0;
@@ -213,7 +223,9 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
               const float4 val =
                   *reinterpret_cast<const float4*>(my_scratch + (rr + sub_row) * PUSH_SCRATCH_STRIDE + col4);
               float* dst = staging + static_cast<size_t>((t / C) * C + static_cast<int>(r)) * p.row_stride + cc + col4;
-              *reinterpret_cast<float4*>(__cluster_map_shared_rank(dst, static_cast<unsigned>(t % C))) = val;
+              const unsigned owner = static_cast<unsigned>(t % C);
+              float* target = owner == r ? dst : static_cast<float*>(__cluster_map_shared_rank(dst, owner));
+              *reinterpret_cast<float4*>(target) = val;
             }
           }
           __syncwarp();

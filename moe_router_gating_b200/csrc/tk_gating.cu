@@ -48,11 +48,12 @@ tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* p
   const int b_boxes = (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES;
   const int scratch = tkg::PUSH_WARPS * tkg::PUSH_SCRATCH_BYTES;
-  int stages = (kMaxDynamicSmem - kSmemReserve - scratch) / stage_bytes;
+  int stages = (kMaxDynamicSmem - kSmemReserve - scratch) / (tkg::KB_PER_STAGE * stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   const int row_stride = round_up(static_cast<int>(E), 32) + 4;
   // the staged partial rows of a tile reuse the ring
-  if (stages < 2 || tkg::BLOCK_M * row_stride * 4 > stages * stage_bytes) return TK_ERR_UNSUPPORTED;
+  if (stages < 2 || tkg::BLOCK_M * row_stride * 4 > stages * tkg::KB_PER_STAGE * stage_bytes)
+    return TK_ERR_UNSUPPORTED;
   const int64_t tiles = (T + tkg::BLOCK_M - 1) / tkg::BLOCK_M;
   plan->variant = TK_VARIANT_SPLIT_H;
   plan->block_m = tkg::BLOCK_M;
@@ -64,7 +65,7 @@ tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* p
   plan->grid = static_cast<int32_t>(tiles * C);
   plan->cluster = C;
   plan->threads = tkg::SPLIT_THREADS;
-  plan->smem_bytes = stages * stage_bytes + scratch + kSmemReserve;
+  plan->smem_bytes = stages * tkg::KB_PER_STAGE * stage_bytes + scratch + kSmemReserve;
   plan->tmem_cols = static_cast<int32_t>(pow2_at_least(round_up(n_pad, 32)));
   return TK_OK;
 }
@@ -117,7 +118,7 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   const int n_pad = pair ? round_up(static_cast<int>(E), 128) : round_up(static_cast<int>(E), 16);
   const int acc_stride = round_up(n_pad, 32);
   const int b_boxes = pair ? n_pad / 2 / tkg::B_BOX_N : (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
-  const int stage_bytes = tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES;
+  const int stage_bytes = tkg::KB_PER_STAGE * (tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES);
   int stages = (kMaxDynamicSmem - kSmemReserve) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return TK_ERR_UNSUPPORTED;
