@@ -238,6 +238,30 @@ def profiled_traffic(wl, digest: str):
     return float(vals["dram_bytes_per_launch"]), os.path.basename(path)
 
 
+# ---------------------------------------------------------------------------
+# multi-rank host logic (one process per GPU; also exercised by CPU gloo tests)
+# ---------------------------------------------------------------------------
+def rank_workload(wl, rank: int):
+    """Each rank gates its own batch of T tokens: the same shapes, another seed."""
+    return workloads.RouterWorkload(wl.name, wl.T, wl.H, wl.E, wl.k, wl.kind, wl.seed + rank,
+                                    wl.dominant, wl.duplicate_pairs)
+
+
+def max_over_ranks(value_ms: float, device, world: int) -> float:
+    """The slowest rank's time (all ranks take part in the reduction)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, elapsed_max_ms: float) -> float:
+    """Whole-job throughput: the tokens all ranks gated, over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (elapsed_max_ms / 1e3)
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -259,8 +283,7 @@ def run_ours(args, wl):
             dist.barrier()
 
     # ---- inputs: seeded host arrays, each rank gates its own token shard ----
-    rank_wl = workloads.RouterWorkload(wl.name, wl.T, wl.H, wl.E, wl.k, wl.kind, wl.seed + rank,
-                                       wl.dominant, wl.duplicate_pairs)
+    rank_wl = rank_workload(wl, rank)
     x_bits = rank_wl.hidden()
     w_bits = rank_wl.gate_weight()
     x_host = workloads.to_torch_bf16(x_bits)
@@ -314,12 +337,9 @@ def run_ours(args, wl):
     if err:
         raise SystemExit(f"device error word {err:#x}: a kernel wait expired during the timed region")
 
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_max_ms = float(t.item())
+    elapsed_max_ms = max_over_ranks(elapsed_ms, dev, world)
     ms_per_step = elapsed_max_ms / args.steps
-    value = world * wl.T * args.steps / (elapsed_max_ms / 1e3)
+    value = job_tokens_per_s(world, wl.T, args.steps, elapsed_max_ms)
 
     # ---- end to end through the host-buffer C-ABI call (pinned host memory) ----
     x_pinned = x_host.pin_memory()
@@ -338,10 +358,7 @@ def run_ours(args, wl):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * wl.T * e2e_steps / (float(te.item()) / 1e3)
+    e2e_value = job_tokens_per_s(world, wl.T, e2e_steps, max_over_ranks(e0.elapsed_time(e1), dev, world))
 
     if world > 1:
         dist.destroy_process_group()
