@@ -7,8 +7,10 @@ never does, and this package imports nothing from the product.
 The arithmetic lives in ``gating_oracle.c`` (plain C, fp64, full per-row sort),
 written from the naive three-step form on the chenxutan.com page, section 4.1
 "MoE Gating": logits = hidden @ gate_weight; top-k of the logits; softmax of
-the k selected values.  Every function of it is pinned by
-``tests/test_oracle_pins.py``; no part is "parity unpinned".
+the k selected values; and in ``route_oracle.c`` (a stable counting sort of the
+token-expert assignments, section 4.2 "MoE Routing").  Every function is pinned
+by ``tests/test_oracle_pins.py`` / ``tests/test_route_oracle.py``; no part is
+"parity unpinned".
 """
 from __future__ import annotations
 
@@ -22,6 +24,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "gating_oracle.c")
+ROUTE_SOURCE = os.path.join(_HERE, "route_oracle.c")
 _LIB = os.path.join(_HERE, "libgating_oracle.so")
 GCC_FLAGS = ["-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off"]
 
@@ -29,17 +32,27 @@ _lock = threading.Lock()
 _libs: dict = {}
 
 
-def compile_oracle(src: str, out: str) -> str:
+def compile_oracle(src: str, out: str, route_src: str = ROUTE_SOURCE) -> str:
+    """Compile a gating-oracle source (possibly a modified copy) with the routing oracle."""
     tmp = out + f".tmp{os.getpid()}"
-    subprocess.check_call(["gcc", *GCC_FLAGS, src, "-o", tmp, "-lm"])
+    subprocess.check_call(["gcc", *GCC_FLAGS, src, route_src, "-o", tmp, "-lm"])
     os.replace(tmp, out)
     return out
 
 
 def build(force: bool = False) -> str:
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(SOURCE):
+    stale = not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(f)
+                                            for f in (SOURCE, ROUTE_SOURCE))
+    if force or stale:
         compile_oracle(SOURCE, _LIB)
     return _LIB
+
+
+@dataclass
+class RouteResult:
+    offsets: np.ndarray       # int32 [E + 1]
+    sorted_slots: np.ndarray  # int32 [n]
+    slot_pos: np.ndarray      # int32 [n]
 
 
 @dataclass
@@ -61,6 +74,8 @@ class Oracle:
         lib.oracle_fused_topk_gating.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_route.argtypes = [vp, i64, ctypes.c_int32, vp, vp, vp]
+        lib.oracle_route.restype = ctypes.c_int
         self._lib = lib
 
     def max_threads(self) -> int:
@@ -87,6 +102,19 @@ class Oracle:
         return OracleResult(scores, scores64, ids, gap, logits)
 
 
+    def route(self, ids: np.ndarray, E: int) -> RouteResult:
+        flat = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+        n = flat.size
+        offsets = np.zeros(E + 1, dtype=np.int32)
+        sorted_slots = np.full(n, -1, dtype=np.int32)
+        slot_pos = np.full(n, -1, dtype=np.int32)
+        rc = self._lib.oracle_route(flat.ctypes.data, n, E, offsets.ctypes.data, sorted_slots.ctypes.data,
+                                    slot_pos.ctypes.data)
+        if rc != 0:
+            raise ValueError(f"oracle_route returned {rc} (n={n} E={E})")
+        return RouteResult(offsets, sorted_slots, slot_pos)
+
+
 def load(lib_path: str | None = None) -> Oracle:
     path = lib_path or build()
     with _lock:
@@ -99,3 +127,8 @@ def fused_topk_gating(hidden_bits: np.ndarray, gate_bits: np.ndarray, k: int,
                       want_logits: bool = False) -> OracleResult:
     """Oracle result for bf16-bit inputs ``hidden[T,H]`` and ``gate_weight[H,E]``."""
     return load().gating(hidden_bits, gate_bits, k, want_logits)
+
+
+def route(ids: np.ndarray, E: int) -> RouteResult:
+    """Oracle routing metadata for expert ids ``[T, k]`` (or flat ``[T*k]``)."""
+    return load().route(ids, E)
