@@ -7,6 +7,10 @@ router, T=65536 tokens, H=7168, E=256 experts, k=8 (hidden 940 MB > L2).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+``--op route`` times the routing metadata (per-expert offsets, the expert-grouped
+order and each assignment's position) of seeded ids of the workload's T x k
+shape; ``--op gating_route`` times gating followed by routing of its ids.
+
 Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one process per GPU)
 every rank gates its own batch of T tokens (token shards, no collective on the
 data path: weak scaling); time is the max over ranks.
@@ -18,7 +22,6 @@ from __future__ import annotations
 
 import argparse
 import datetime
-import hashlib
 import json
 import os
 import statistics
@@ -56,6 +59,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (profiling cases)")
+    ap.add_argument("--op", default="gating", choices=("gating", "route", "gating_route"),
+                    help="gating (default); route: routing metadata of the workload's T x k ids; "
+                         "gating_route: both, chained on the device")
     return ap.parse_args()
 
 
@@ -211,14 +217,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 def kernel_source_digest() -> str:
     from moe_router_gating_b200 import build as tkbuild
-    h = hashlib.sha256()
-    for p in tkbuild._inputs():
-        if p.endswith(".py"):
-            continue
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
-            h.update(f.read())
-    return h.hexdigest()[:16]
+    return tkbuild.gating_kernel_digest()
 
 
 def profiled_traffic(wl, digest: str):
@@ -430,11 +429,148 @@ def run_ours(args, wl):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# routing metadata (--op route / gating_route), one GPU
+# ---------------------------------------------------------------------------
+ROUTE_METRIC = "routing metadata tokens/s"
+CHAIN_METRIC = "gating + routing tokens/s"
+
+
+def route_bytes(T: int, k: int, E: int) -> int:
+    """ids read once; sorted_slots, slot_pos and offsets written once."""
+    return 12 * T * k + 4 * (E + 1)
+
+
+def time_route_oracle(T, k, E, seconds: float):
+    import oracle
+    orc = oracle.load()
+    ids = workloads.expert_ids(T, k, E, seed=0)
+    reps, dt = 0, 0.0
+    t0 = time.perf_counter()
+    while dt < seconds:
+        orc.route(ids, E)
+        reps += 1
+        dt = time.perf_counter() - t0
+    return T * reps / dt, reps, dt
+
+
+def run_route_ours(args, wl):
+    import torch
+
+    import moe_router_gating_b200 as tk
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--op route runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T, k, E = wl.T, wl.k, wl.E
+    chain = args.op == "gating_route"
+    stream = torch.cuda.current_stream(dev)
+    ids_host = torch.from_numpy(workloads.expert_ids(T, k, E, seed=0))
+    ids = ids_host.to(dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sorted_slots = torch.empty(T * k, dtype=torch.int32, device=dev)
+    slot_pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if chain:
+        x = workloads.to_torch_bf16(wl.hidden()).to(dev)
+        w = workloads.to_torch_bf16(wl.gate_weight()).to(dev)
+        scores = torch.empty((T, k), dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        if chain:
+            tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream)
+        tk.route(ids, E, offsets, sorted_slots, slot_pos, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    tk.device_error(clear=True)
+    sampler = ClockSampler(0)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with sampler:
+        for a, b in evs:
+            flush.zero_()  # ids (and the gate) would otherwise stay in L2 between steps
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+    per = [a.elapsed_time(b) for a, b in evs]
+    if tk.device_error(clear=True):
+        raise SystemExit("a kernel wait expired during the timed region")
+    elapsed_ms = sum(per)
+    ms_per_step = elapsed_ms / args.steps
+    value = T * args.steps / (elapsed_ms / 1e3)
+
+    # end to end: pinned host ids -> device, route, the three outputs -> pinned host
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    ids_pinned = ids_host.pin_memory()
+    outs_host = [torch.empty(t.shape, dtype=torch.int32).pin_memory() for t in (offsets, sorted_slots, slot_pos)]
+
+    def e2e_step():
+        ids.copy_(ids_pinned, non_blocking=True)
+        tk.route(ids, E, offsets, sorted_slots, slot_pos, stream=stream)
+        for h, d in zip(outs_host, (offsets, sorted_slots, slot_pos)):
+            h.copy_(d, non_blocking=True)
+
+    e2e_value = None
+    if not chain:
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_value = T * e2e_steps / (e0.elapsed_time(e1) / 1e3)
+
+    peaks, peak_src = load_peaks()
+    bytes_alg = route_bytes(T, k, E)
+    plan = tk.route_plan(T, k, E, torch.cuda.get_device_properties(dev).multi_processor_count)
+    line = {
+        "metric": CHAIN_METRIC if chain else ROUTE_METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int32" if not chain else "bf16", "data": "synthetic",
+        "config": {"workload": (workload_desc(wl) if chain else
+                                f"route of {wl.name}-shaped ids: T={T} k={k} E={E}, uniform seeded ids, "
+                                "k distinct per token"),
+                   "T": T, "k": k, "E": E,
+                   "l2": "L2 flushed (256 MB write) before every timed step; each step timed alone",
+                   "launch": plan},
+        "gpu_launches": args.steps * (3 if chain else 2),
+        "clocks": sampler.summary(),
+    }
+    if not chain:
+        ach = bytes_alg / (ms_per_step / 1e3) / 1e9
+        line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                            "peak_source": f"{peak_src}; copy GB/s (of measured)",
+                            "algorithmic_bytes_per_step": bytes_alg,
+                            "note": "two launches per step (count, then scatter); time of the pair"}
+        line["e2e"] = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 4 * T * k,
+                       "d2h_bytes_per_step": 4 * (E + 1) + 8 * T * k,
+                       "path": "pinned host ids -> device, tk_gating_route, three outputs -> pinned host"}
+        if not args.no_cpu_baseline:
+            v, reps, dt = time_route_oracle(T, k, E, min(args.cpu_seconds, 5.0))
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": f"whole workload, {reps} calls in {dt:.1f} s (single-thread C)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     wl = workloads.WORKLOADS[args.workload]
     if args.tokens is not None:
         wl = wl.with_T(args.tokens)
+    if args.op != "gating":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers --op gating only"}))
+            return 0
+        return run_route_ours(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

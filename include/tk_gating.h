@@ -22,7 +22,8 @@
  * Conventions for every entry point below:
  *   - Pointers marked "device" are CUDA global-memory addresses on the current
  *     device; the caller allocates and owns every buffer.  The library keeps no
- *     per-call state and allocates no device memory.
+ *     per-call state.  Only tk_gating_route allocates device memory: a
+ *     stream-ordered workspace that it frees on the same stream.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls are asynchronous: they return once the work is enqueued.  Launch
  *     failures return TK_ERR_CUDA; faults inside a kernel surface at the
@@ -156,6 +157,83 @@ TK_API tk_status tk_gating_device_error(uint32_t* word, int32_t clear);
  * below 1000 are rejected with TK_ERR_INVALID_ARG.
  */
 TK_API tk_status tk_gating_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/*
+ * ---------------------------------------------------------------------------
+ * Routing metadata (the local part of MoE dispatch).
+ *
+ * The operation (chenxutan.com, "TileKernels 深度解析", section 4.2 "MoE
+ * Routing"): dispatch sends every token to the experts its expert_ids row
+ * names, and combine puts the experts' results back with the indices dispatch
+ * returned.  Before any exchange, the T*k token-expert assignments have to be
+ * grouped by expert.  For assignment s = t*k + j (token t, rank j) with expert
+ * e = ids[s]:
+ *
+ *   offsets[e]       number of assignments to experts below e (exclusive
+ *                    prefix sum of the per-expert counts); offsets[E] is the
+ *                    number placed, so expert e owns positions
+ *                    [offsets[e], offsets[e+1]);
+ *   sorted_slots[p]  the assignment s at position p of the grouped order;
+ *                    inside an expert the assignments keep ascending s (a
+ *                    stable order: the result is unique and deterministic);
+ *   slot_pos[s]      the position p of assignment s (the inverse of
+ *                    sorted_slots; the page's dispatch_indices in this
+ *                    library's reading).
+ *
+ * An id outside [0, E) is neither counted nor placed: its slot_pos is -1 and
+ * offsets[E] falls short of T*k by the number of such ids; the positions
+ * offsets[E] .. T*k-1 of sorted_slots are then not written.
+ * ---------------------------------------------------------------------------
+ */
+#define TK_ROUTE_MAX_EXPERTS 1024
+
+/* The launches tk_gating_route makes (host logic, no GPU needed). */
+typedef struct {
+  int32_t ctas;               /* CTAs of each kernel; 1 = a single kernel and no workspace */
+  int32_t threads;            /* threads per CTA */
+  int64_t warp_slots;         /* assignments per warp range (a multiple of 32) */
+  int64_t workspace_bytes;    /* device workspace: ctas x round_up(E, 4) int32 counts, 0 when ctas == 1 */
+  int32_t count_smem_bytes;   /* dynamic shared memory of the counting kernel */
+  int32_t scatter_smem_bytes; /* dynamic shared memory of the placing kernel */
+} tk_route_plan;
+
+/*
+ * tk_gating_route -- routing metadata of ids[T, k].
+ *
+ *   ids           device, int32 [T, k] row-major (for example the ids output
+ *                 of tk_gating_fused_topk); read only.
+ *   T, k          tokens (T >= 0) and assignments per token (k >= 1);
+ *                 T * k < 2^31.
+ *   E             experts, 1 <= E <= 1024.
+ *   offsets       device, out int32 [E + 1].
+ *   sorted_slots  device, out int32 [T * k].
+ *   slot_pos      device, out int32 [T, k].
+ *   stream        cudaStream_t (void*), may be NULL.
+ *
+ * Up to 4096 assignments: one kernel launch on `stream`, no workspace.
+ * Beyond: two launches, the second a programmatic dependent launch of the
+ * first, with a workspace of tk_route_plan.workspace_bytes (at most
+ * 148 x 1024 x 4 bytes on a B200) that the call takes with cudaMallocAsync
+ * from the device's default memory pool and releases with cudaFreeAsync after
+ * the launches, both on `stream`.  T * k == 0 is valid: offsets is set to
+ * zeros and ids, sorted_slots and slot_pos may then be NULL.
+ *
+ * Errors:
+ *   TK_ERR_INVALID_ARG   T < 0, k < 1, E < 1, offsets NULL, or another
+ *                        pointer NULL when T * k > 0;
+ *   TK_ERR_UNSUPPORTED   E > 1024, T * k >= 2^31, or the device is not sm_100;
+ *   TK_ERR_ALIGNMENT     a pointer is not 4-byte aligned;
+ *   TK_ERR_CUDA          the workspace allocation or a launch failed.
+ */
+TK_API tk_status tk_gating_route(const int32_t* ids, int64_t T, int32_t k, int32_t E, int32_t* offsets,
+                                 int32_t* sorted_slots, int32_t* slot_pos, void* stream);
+
+/*
+ * tk_gating_route_plan -- fill *plan with the launches tk_gating_route makes
+ * for (T, k, E) on a device with `num_sms` SMs.  Validates sizes like
+ * tk_gating_route.  Makes no CUDA call.
+ */
+TK_API tk_status tk_gating_route_plan(int64_t T, int32_t k, int32_t E, int32_t num_sms, tk_route_plan* plan);
 
 /* Static string for a status code. */
 TK_API const char* tk_gating_status_string(tk_status status);

@@ -28,11 +28,15 @@ from ._binding import (  # noqa: F401
     library,
     library_path,
     make_plan,
+    route,
+    route_plan,
+    route_ptr,
     set_wait_timeout_ns,
     status_string,
 )
 
 __all__ = [
-    "fused_topk_gating", "fused_topk_gating_host", "fused_topk_gating_ptr", "make_plan", "device_error",
+    "fused_topk_gating", "fused_topk_gating_host", "fused_topk_gating_ptr", "make_plan", "route", "route_plan",
+    "route_ptr", "device_error",
     "set_wait_timeout_ns", "status_string", "TkGatingError", "library", "library_path",
 ]

@@ -34,6 +34,12 @@ class _Plan(ctypes.Structure):
         "threads", "smem_bytes", "tmem_cols", "num_half_tiles")]
 
 
+class _RoutePlan(ctypes.Structure):
+    _fields_ = [("ctas", ctypes.c_int32), ("threads", ctypes.c_int32), ("warp_slots", ctypes.c_int64),
+                ("workspace_bytes", ctypes.c_int64), ("count_smem_bytes", ctypes.c_int32),
+                ("scatter_smem_bytes", ctypes.c_int32)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -58,6 +64,10 @@ def library() -> ctypes.CDLL:
             lib.tk_gating_device_error.restype = ctypes.c_int
             lib.tk_gating_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
             lib.tk_gating_set_wait_timeout_ns.restype = ctypes.c_int
+            lib.tk_gating_route.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
+            lib.tk_gating_route.restype = ctypes.c_int
+            lib.tk_gating_route_plan.argtypes = [i64, i32, i32, i32, ctypes.POINTER(_RoutePlan)]
+            lib.tk_gating_route_plan.restype = ctypes.c_int
             lib.tk_gating_status_string.argtypes = [ctypes.c_int]
             lib.tk_gating_status_string.restype = ctypes.c_char_p
             _lib = lib
@@ -162,3 +172,45 @@ def device_error(clear: bool = True) -> int:
 
 def set_wait_timeout_ns(timeout_ns: int) -> None:
     _check(library().tk_gating_set_wait_timeout_ns(int(timeout_ns)), "tk_gating_set_wait_timeout_ns")
+
+
+def route_plan(T: int, k: int, E: int, num_sms: int = 148) -> dict:
+    """The launches ``route`` would make (host logic only; no GPU needed)."""
+    p = _RoutePlan()
+    _check(library().tk_gating_route_plan(T, k, E, num_sms, ctypes.byref(p)), "tk_gating_route_plan")
+    return {name: getattr(p, name) for name, _ in _RoutePlan._fields_}
+
+
+def route_ptr(ids: int, T: int, k: int, E: int, offsets: int, sorted_slots: int, slot_pos: int,
+              stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the tk_status."""
+    return int(library().tk_gating_route(ids, T, k, E, offsets, sorted_slots, slot_pos, stream))
+
+
+def route(ids, num_experts: int, offsets=None, sorted_slots=None, slot_pos=None, stream=None):
+    """Routing metadata of expert ids ``[T, k]`` (CUDA int32, contiguous):
+    ``(offsets[E+1], sorted_slots[T*k], slot_pos[T,k])``, all int32 -- the
+    assignments grouped by expert, ascending inside an expert.  Output tensors
+    may be passed in.  The launches go on ``stream`` (default: the current
+    torch stream)."""
+    import torch
+    if ids.dtype != torch.int32 or ids.dim() != 2 or not ids.is_cuda or not ids.is_contiguous():
+        raise ValueError("ids must be a contiguous CUDA int32 [T, k] tensor")
+    T, k = ids.shape
+    E = int(num_experts)
+    dev = ids.device
+    if offsets is None:
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if sorted_slots is None:
+        sorted_slots = torch.empty(T * k, dtype=torch.int32, device=dev)
+    if slot_pos is None:
+        slot_pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    for name, t, n in (("offsets", offsets, E + 1), ("sorted_slots", sorted_slots, T * k),
+                       ("slot_pos", slot_pos, T * k)):
+        if t.dtype != torch.int32 or t.numel() != n or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous int32 tensor of {n} elements on {dev}")
+    with torch.cuda.device(dev):
+        st = library().tk_gating_route(ids.data_ptr(), T, k, E, offsets.data_ptr(), sorted_slots.data_ptr(),
+                                       slot_pos.data_ptr(), _stream_handle(stream, dev))
+    _check(st, "tk_gating_route")
+    return offsets, sorted_slots, slot_pos

@@ -7,7 +7,9 @@ the public header is newer than the library.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -41,6 +43,29 @@ def sources() -> list[str]:
 def _inputs() -> list[str]:
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
         sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [os.path.abspath(__file__)]
+
+
+# Sources that compile into the fused gating kernels (not the routing kernels).
+GATING_KERNEL_SOURCES = ("tk_gating.cu", "gating_row_tiles.cuh", "gating_split_h.cuh", "sm100_ptx.cuh",
+                         "topk_epilogue.cuh", "topk_merge.cuh")
+
+
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines (string literals here hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
+def gating_kernel_digest() -> str:
+    """Digest of the gating kernels' code (comments ignored): a profile measured on
+    these kernels stays valid while it is unchanged."""
+    h = hashlib.sha256()
+    for name in GATING_KERNEL_SOURCES:
+        with open(os.path.join(CSRC, name)) as f:
+            h.update(name.encode())
+            h.update(_code_only(f.read()).encode())
+    return h.hexdigest()[:16]
 
 
 def is_stale() -> bool:

@@ -13,7 +13,6 @@ and the digest of the kernel sources, which bench.py reports as the roofline's
 from __future__ import annotations
 
 import csv
-import hashlib
 import os
 import sys
 from collections import OrderedDict
@@ -41,16 +40,9 @@ REPORT_METRICS = [
 
 
 def kernel_source_digest() -> str:
-    """Same digest as bench.py: the kernel sources and the public header."""
+    """Same digest as bench.py: the gating kernels' code, comments ignored."""
     from moe_router_gating_b200 import build as tkbuild
-    h = hashlib.sha256()
-    for p in tkbuild._inputs():
-        if p.endswith(".py"):
-            continue
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
-            h.update(f.read())
-    return h.hexdigest()[:16]
+    return tkbuild.gating_kernel_digest()
 
 
 def _rows(path):

@@ -174,6 +174,26 @@ DECODE = tuple(RouterWorkload(f"decode_T{t}", t, 7168, 256, 8) for t in DECODE_T
 WORKLOADS = {w.name: w for w in (TINY, DEEPSEEK, SKEW, TRAIN) + DECODE}
 
 
+def expert_ids(T: int, k: int, E: int, seed: int, kind: str = "uniform") -> np.ndarray:
+    """Seeded int32 ``[T, k]`` expert ids, k distinct per row (as a router emits).
+
+    ``uniform``: every expert equally likely.  ``skew``: expert popularity drawn
+    from a Dirichlet(0.3) (a few hot experts, a long cold tail), rows sampled
+    without replacement by the Gumbel-top-k rule.  Inputs for the routing
+    metadata only; nothing of the routing itself is computed here.
+    """
+    if not 1 <= k <= E:
+        raise ValueError(f"need 1 <= k <= E, got k={k} E={E}")
+    rng = np.random.default_rng(seed)
+    keys = rng.random((T, E), dtype=np.float32)
+    if kind == "skew":
+        logp = np.log(rng.dirichlet(np.full(E, 0.3)) + 1e-30).astype(np.float32)
+        keys = logp[None, :] - np.log(-np.log(np.maximum(keys, np.float32(1e-12))))
+    elif kind != "uniform":
+        raise ValueError(f"unknown kind {kind!r}")
+    return np.argpartition(-keys, k - 1, axis=1)[:, :k].astype(np.int32) if T else np.zeros((0, k), np.int32)
+
+
 def to_torch_bf16(bits: np.ndarray):
     """View a uint16 bf16-bit array as a CPU ``torch.bfloat16`` tensor (no copy)."""
     import torch
