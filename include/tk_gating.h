@@ -235,6 +235,37 @@ TK_API tk_status tk_gating_route(const int32_t* ids, int64_t T, int32_t k, int32
  */
 TK_API tk_status tk_gating_route_plan(int64_t T, int32_t k, int32_t E, int32_t num_sms, tk_route_plan* plan);
 
+/*
+ * tk_gating_route_static -- tk_gating_route without any allocation.
+ *
+ * The pages have no counterpart: this is a property of this library's
+ * interface.  It is for callers that cannot let the library allocate device
+ * memory: a process whose device memory is reserved up front by its own
+ * allocator (a pool allocation could then fail in the middle of a run), or
+ * code that must not enter the driver's allocator at all (growing a memory
+ * pool maps new memory).  The result is the same as tk_gating_route's; the
+ * counts table that tk_gating_route takes from cudaMallocAsync lives here in
+ * a fixed device array of TK_ROUTE_STATIC_SCRATCH_BYTES, one per device.
+ *
+ *   Arguments, layouts and the other errors as tk_gating_route.
+ *   TK_ERR_UNSUPPORTED also when the launch needs more scratch than the array
+ *   holds (tk_route_plan.workspace_bytes > TK_ROUTE_STATIC_SCRATCH_BYTES):
+ *   never for E <= 440 on a device of at most 148 SMs; for larger E while the
+ *   plan's ctas x round_up(E, 4) x 4 bytes fit (E = 1024: up to 262144
+ *   assignments).  Nothing is written then.
+ *   TK_ERR_CUDA when the array's device address cannot be obtained.
+ *
+ * Set-up: the first call made with a device current looks up the array's
+ * device address on that device (and loads the library's kernels there if
+ * that has not happened yet); make that first call before any stream capture.
+ * Calls that overlap on one device (issued to different streams, or from
+ * different host threads, without ordering between them) share the one
+ * array and race: order them, for example by issuing them to one stream.
+ */
+#define TK_ROUTE_STATIC_SCRATCH_BYTES (256 * 1024)
+TK_API tk_status tk_gating_route_static(const int32_t* ids, int64_t T, int32_t k, int32_t E, int32_t* offsets,
+                                        int32_t* sorted_slots, int32_t* slot_pos, void* stream);
+
 /* Static string for a status code. */
 TK_API const char* tk_gating_status_string(tk_status status);
 

@@ -31,6 +31,7 @@ from ._binding import (  # noqa: F401
     route,
     route_plan,
     route_ptr,
+    route_static_ptr,
     set_wait_timeout_ns,
     status_string,
 )

@@ -66,6 +66,8 @@ def library() -> ctypes.CDLL:
             lib.tk_gating_set_wait_timeout_ns.restype = ctypes.c_int
             lib.tk_gating_route.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
             lib.tk_gating_route.restype = ctypes.c_int
+            lib.tk_gating_route_static.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
+            lib.tk_gating_route_static.restype = ctypes.c_int
             lib.tk_gating_route_plan.argtypes = [i64, i32, i32, i32, ctypes.POINTER(_RoutePlan)]
             lib.tk_gating_route_plan.restype = ctypes.c_int
             lib.tk_gating_status_string.argtypes = [ctypes.c_int]
@@ -214,3 +216,10 @@ def route(ids, num_experts: int, offsets=None, sorted_slots=None, slot_pos=None,
                                        slot_pos.data_ptr(), _stream_handle(stream, dev))
     _check(st, "tk_gating_route")
     return offsets, sorted_slots, slot_pos
+
+
+def route_static_ptr(ids: int, T: int, k: int, E: int, offsets: int, sorted_slots: int, slot_pos: int,
+                     stream: int = 0) -> int:
+    """Raw C-ABI call of the no-allocation routing entry point (integer device
+    pointers); returns the tk_status."""
+    return int(library().tk_gating_route_static(ids, T, k, E, offsets, sorted_slots, slot_pos, stream))

@@ -173,6 +173,43 @@ tk_status route_checked(const int32_t* ids, int64_t T, int32_t k, int32_t E, int
   return route_plan_impl(T, k, E, dev->num_sms, pl);
 }
 
+// ---- tk_gating_route_static: the counts table in a fixed device array ----
+//
+// For callers that cannot let the library allocate device memory.  The
+// several-CTA path needs G x round_up(E, 4) int32 of scratch (the counts
+// table); here it lives in this file-scope array instead of a stream-ordered
+// allocation.  Every word the placing kernel reads is written by the counting
+// kernel of the same call first, so nothing in it has to start at zero.  One
+// array per device serves every call: calls that overlap on the device (other
+// streams, other host threads) race on it.
+static __device__ __align__(256) int32_t g_route_static_scratch[TK_ROUTE_STATIC_SCRATCH_BYTES / 4];
+
+struct StaticScratch {
+  bool ready = false;
+  int32_t* ptr = nullptr;  // device address of g_route_static_scratch on that device
+};
+
+StaticScratch g_static_scratch[kMaxDevices];
+std::mutex g_static_scratch_mutex;
+
+// Set-up on the first call made with a device current: the array's device
+// address (cudaGetSymbolAddress may load the module onto the device).
+int32_t* static_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  StaticScratch& sc = g_static_scratch[dev];
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (sc.ready) return sc.ptr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return nullptr;  // not cached: a later call retries
+  }
+  sc.ptr = static_cast<int32_t*>(p);
+  sc.ready = true;
+  return sc.ptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -199,6 +236,19 @@ tk_status tk_gating_route(const int32_t* ids, int64_t T, int32_t k, int32_t E, i
                     slot_pos, s);
   if (cudaFreeAsync(ws, s) != cudaSuccess && st == TK_OK) st = TK_ERR_CUDA;
   return st;
+}
+
+tk_status tk_gating_route_static(const int32_t* ids, int64_t T, int32_t k, int32_t E, int32_t* offsets,
+                                 int32_t* sorted_slots, int32_t* slot_pos, void* stream) {
+  const RouteDevice* dev = nullptr;
+  tk_route_plan pl;
+  tk_status st = route_checked(ids, T, k, E, offsets, sorted_slots, slot_pos, &dev, &pl);
+  if (st != TK_OK) return st;
+  if (pl.workspace_bytes > TK_ROUTE_STATIC_SCRATCH_BYTES) return TK_ERR_UNSUPPORTED;
+  int32_t* scratch = static_scratch();
+  if (scratch == nullptr) return TK_ERR_CUDA;
+  return launch_route(pl, ids, T * static_cast<int64_t>(k), E, pl.workspace_bytes > 0 ? scratch : nullptr, offsets,
+                      sorted_slots, slot_pos, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
