@@ -57,8 +57,8 @@ typedef enum {
 } tk_status;
 
 /* Limits of the fused kernels. */
-#define TK_GATING_MAX_EXPERTS 256
-#define TK_GATING_MAX_TOPK 16
+#define TK_GATING_MAX_EXPERTS 512
+#define TK_GATING_MAX_TOPK 32
 
 /*
  * tk_gating_fused_topk -- the fused gating operator.
@@ -68,8 +68,8 @@ typedef enum {
  *                `hidden_states @ gate_weight`; expert e is column e).
  *   T            tokens, T >= 0.  T == 0 returns TK_OK and launches nothing.
  *   H            hidden size, H >= 8 and H % 8 == 0 (16-byte row pitch).
- *   E            experts, 16 <= E <= 256 and E % 8 == 0.
- *   k            experts kept per token, 1 <= k <= min(E, 16).
+ *   E            experts, 16 <= E <= 512 and E % 8 == 0.
+ *   k            experts kept per token, 1 <= k <= min(E, 32).
  *   scores       device, out fp32 [T, k] row-major.
  *   ids          device, out int32 [T, k] row-major.
  *   stream       cudaStream_t (void*), may be NULL.
@@ -77,7 +77,7 @@ typedef enum {
  * Errors:
  *   TK_ERR_INVALID_ARG   T < 0, H < 1, E < 1, k < 1, k > E, or a null pointer
  *                        when T > 0;
- *   TK_ERR_UNSUPPORTED   H or E not a multiple of 8, E < 16, E > 256, k > 16,
+ *   TK_ERR_UNSUPPORTED   H or E not a multiple of 8, E < 16, E > 512, k > 32,
  *                        T >= 2^31 - 128, or the current device is not sm_100;
  *   TK_ERR_ALIGNMENT     a pointer is not 16-byte aligned;
  *   TK_ERR_CUDA          a CUDA call (device query, descriptor encode, launch)
@@ -120,17 +120,19 @@ typedef enum {
 typedef struct {
   int32_t variant;      /* tk_variant */
   int32_t block_m;      /* tokens per tile */
-  int32_t n_pad;        /* MMA N: E rounded up to a multiple of 16 */
+  int32_t n_pad;        /* MMA N over all experts: E rounded up to a multiple of 16 (CTA pairs: of
+                           128); one MMA per chunk of up to 256 experts and K step */
   int32_t num_tiles;    /* full tiles of block_m tokens (all of T unless num_half_tiles > 0) */
   int32_t k_blocks;     /* ceil(H / 64) */
   int32_t split_h;      /* CTAs sharing one tile's H range (1 = none) */
-  int32_t stages;       /* shared-memory ring depth (row tiles: stages of two 64-wide K slices) */
+  int32_t stages;       /* shared-memory ring depth, in stages of slices_per_stage K slices */
   int32_t grid;         /* CTAs launched */
   int32_t cluster;      /* CTAs per cluster */
   int32_t threads;      /* threads per CTA */
   int32_t smem_bytes;   /* dynamic shared memory per CTA */
   int32_t tmem_cols;    /* tensor-memory columns allocated per CTA */
   int32_t num_half_tiles; /* CTA pairs: 128-token tiles after the full ones (balanced last round) */
+  int32_t slices_per_stage; /* 64-wide K slices per ring stage */
 } tk_gating_plan;
 
 /*

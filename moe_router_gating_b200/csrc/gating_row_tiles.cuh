@@ -11,6 +11,11 @@
 //   both CTAs' shared memory and write each CTA's 128 rows x N logits into its
 //   own tensor memory.  Per CTA this halves the gate bytes each tile pulls from
 //   L2 compared with CG = 1.
+//   More than 256 experts (up to 512): the MMA N is split into chunks of at
+//   most 256 columns, one tcgen05.mma per chunk and K step, chunk c
+//   accumulating experts [256c, 256c + N_c) in tensor-memory columns from 256c;
+//   in a pair each CTA holds half of every chunk's gate columns.  The
+//   accumulator then fills tensor memory, so it is single-buffered.
 //   Balanced tail: when the last round of 256-token tiles would leave pairs
 //   idle, the remaining rows run as 128-token "half" tiles (M = 128 pair MMAs,
 //   64 rows per CTA): half the MMA cycles and three quarters of the bytes of a
@@ -55,10 +60,14 @@ constexpr int NUM_EPI_WARPS = 4;
 constexpr int KB_PER_STAGE = 2;                         // 64-wide K slices per ring stage
 constexpr int ROW_TILE_THREADS = 64 + NUM_EPI_WARPS * 32;
 
+constexpr int N_CHUNK = 256;                            // MMA N per instruction (chunk of experts)
+
 struct RowTileParams {
   int32_t T, H, E, k;
-  int32_t n_pad;        // MMA N (CG=1: E rounded up to 16; CG=2: 128 or 256)
-  int32_t acc_stride;   // TMEM columns between the two accumulator buffers
+  int32_t n_pad;        // total MMA N (CG=1: E rounded up to 16; CG=2: a multiple of 128, <= 512)
+  int32_t n_chunks;     // ceil(n_pad / 256): MMAs per K step
+  int32_t acc_stride;   // TMEM columns between accumulator buffers
+  int32_t acc_bufs;     // accumulator buffers in TMEM (2, or 1 when n_pad > 256)
   int32_t num_tiles;    // full tiles of BLOCK_M * CG rows, starting at row 0
   int32_t num_half;     // pairs only: half tiles of BLOCK_M rows after the full tiles
   int32_t k_blocks;
@@ -85,6 +94,17 @@ __device__ __forceinline__ uint64_t a_desc_k_slice(uint32_t a_stage_addr, int kk
 }
 __device__ __forceinline__ uint64_t b_desc_k_slice(uint32_t b_stage_addr, int kk) {
   return smem_desc_sw128(b_stage_addr + kk * (UMMA_K / 8) * 1024, B_BOX_BYTES, 1024);
+}
+
+// Width of MMA chunk c (all but the last are N_CHUNK wide).
+__device__ __forceinline__ int chunk_n(const RowTileParams& p, int c) {
+  return c + 1 < p.n_chunks ? N_CHUNK : p.n_pad - N_CHUNK * (p.n_chunks - 1);
+}
+
+// Gate boxes (64 experts each) of chunk c that one CTA stages per K slice.
+template <int CG>
+__device__ __forceinline__ int chunk_boxes(const RowTileParams& p, int c) {
+  return (chunk_n(p, c) / CG + B_BOX_N - 1) / B_BOX_N;
 }
 
 // The i-th tile of a CTA (or pair) `unit` out of `units`: full tiles round-robin,
@@ -192,7 +212,11 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       // ---------------- TMA producer ----------------
       const uint64_t pol_x = l2_policy_evict_first();  // hidden: streamed once
       const uint64_t pol_w = l2_policy_evict_last();   // gate: re-read by every tile
-      const int b_col0 = static_cast<int>(rank) * p.b_boxes * B_BOX_N;  // this CTA's gate columns
+      // gate box j of a K slice starts at column j * 64 + (j < bpc0 ? col_a : col_b): this
+      // CTA's share of chunk 0 (bpc0 boxes), then of chunk 1 (starting at expert 256)
+      const int bpc0 = chunk_boxes<CG>(p, 0);
+      const int col_a = static_cast<int>(rank) * (chunk_n(p, 0) / CG);
+      const int col_b = p.n_chunks > 1 ? N_CHUNK + static_cast<int>(rank) * (chunk_n(p, 1) / CG) - bpc0 * B_BOX_N : 0;
       uint32_t stage = 0, phase = 0;
       int issued = 0;
       bool ok = true;
@@ -217,13 +241,13 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
               const uint32_t bar = map_shared_rank(smem_u32(&full[stage]), 0);
               tma_load_2d_pair(sA + slot * A_STAGE_BYTES, map_a, bar, k0, row0, pol_x);
               for (int j = 0; j < p.b_boxes; ++j)
-                tma_load_2d_pair(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, bar, b_col0 + j * B_BOX_N, k0,
-                                 pol_w);
+                tma_load_2d_pair(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, bar,
+                                 j * B_BOX_N + (j < bpc0 ? col_a : col_b), k0, pol_w);
             } else {
               tma_load_2d(sA + slot * A_STAGE_BYTES, &map_x, &full[stage], k0, row0, pol_x);
               for (int j = 0; j < p.b_boxes; ++j)
-                tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], b_col0 + j * B_BOX_N, k0,
-                            pol_w);
+                tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage],
+                            j * B_BOX_N + (j < bpc0 ? col_a : col_b), k0, pol_w);
             }
           }
           ++issued;
@@ -252,16 +276,27 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer ----------------
-      const uint32_t idesc_full = idesc_bf16_f32(BLOCK_M * CG, p.n_pad, false, true);
-      const uint32_t idesc_half = idesc_bf16_f32(BLOCK_M, p.n_pad, false, true);  // pairs: 64 rows per CTA
+      // per chunk: instruction descriptor (full and half tiles) and the offset of
+      // its gate boxes within a K slice
+      uint32_t idesc_full[2], idesc_half[2], b_off[2];
+#pragma unroll
+      for (int c = 0, box = 0; c < 2; ++c) {
+        const int nc = c < p.n_chunks ? chunk_n(p, c) : N_CHUNK;
+        idesc_full[c] = idesc_bf16_f32(BLOCK_M * CG, nc, false, true);
+        idesc_half[c] = idesc_bf16_f32(BLOCK_M, nc, false, true);  // pairs: 64 rows per CTA
+        b_off[c] = static_cast<uint32_t>(box * B_BOX_BYTES);
+        if (c < p.n_chunks) box += chunk_boxes<CG>(p, c);
+      }
+      const bool two_chunks = p.n_chunks > 1;
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
       TileWork w;
       for (; ok && tile_work<CG>(p, unit, units, local, w); ++local) {
-        const uint32_t buf = local & 1;
-        const uint32_t acc_phase = (local >> 1) & 1;
-        const uint32_t idesc = w.half ? idesc_half : idesc_full;
+        const uint32_t buf = static_cast<uint32_t>(local % p.acc_bufs);
+        const uint32_t acc_phase = static_cast<uint32_t>(local / p.acc_bufs) & 1;
+        const uint32_t id0 = w.half ? idesc_half[0] : idesc_full[0];
+        const uint32_t id1 = w.half ? idesc_half[1] : idesc_full[1];
         if (!mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + buf * p.acc_stride;
@@ -276,13 +311,30 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
             const int slot = stage * KB_PER_STAGE + sub;
             const uint32_t a_addr = smem_u32(sA + slot * A_STAGE_BYTES);
             const uint32_t b_addr = smem_u32(sB + slot * p.b_boxes * B_BOX_BYTES);
+            // the chunk count is loop-invariant: one branch per slice, none per MMA
+            // (extra work between MMAs measurably slows the issue loop)
+            if (two_chunks) {
 #pragma unroll
-            for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
-              const uint32_t accumulate = ((kb + sub) | kk) != 0;
-              if constexpr (kPair)
-                umma_bf16_pair(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc, accumulate);
-              else
-                umma_bf16(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc, accumulate);
+              for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
+                const uint32_t accumulate = ((kb + sub) | kk) != 0;
+                const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
+                if constexpr (kPair) {
+                  umma_bf16_pair(d_tmem, a_desc, b_desc_k_slice(b_addr, kk), id0, accumulate);
+                  umma_bf16_pair(d_tmem + N_CHUNK, a_desc, b_desc_k_slice(b_addr + b_off[1], kk), id1, accumulate);
+                } else {
+                  umma_bf16(d_tmem, a_desc, b_desc_k_slice(b_addr, kk), id0, accumulate);
+                  umma_bf16(d_tmem + N_CHUNK, a_desc, b_desc_k_slice(b_addr + b_off[1], kk), id1, accumulate);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
+                const uint32_t accumulate = ((kb + sub) | kk) != 0;
+                if constexpr (kPair)
+                  umma_bf16_pair(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), id0, accumulate);
+                else
+                  umma_bf16(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), id0, accumulate);
+              }
             }
           }
           // frees the stage (in both CTAs of a pair) once these MMAs have read it
@@ -317,29 +369,39 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     int local = 0;
     TileWork w;
     for (; tile_work<CG>(p, unit, units, local, w); ++local) {
-      const uint32_t buf = local & 1;
-      const uint32_t acc_phase = (local >> 1) & 1;
+      const uint32_t buf = static_cast<uint32_t>(local % p.acc_bufs);
+      const uint32_t acc_phase = static_cast<uint32_t>(local / p.acc_bufs) & 1;
       bool ok = mbar_wait(&acc_full[buf], acc_phase, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
 
-      // full tile: one row per thread over all experts; half tile: lanes 0..63
-      // hold experts [0, N/2) and lanes 64..127 experts [N/2, N) of 64 rows
+      // full tile: one row per thread, TMEM column e = expert e; half tile:
+      // per chunk c, lanes 0..63 hold experts [256c, 256c + N_c/2) and lanes
+      // 64..127 experts [256c + N_c/2, 256c + N_c) of 64 rows, in columns from 256c
       const bool upper = w.half && quad >= 2;
-      const int col_base = upper ? p.n_pad / 2 : 0;
-      const int ncols = w.half ? min(p.n_pad / 2, p.E - col_base) : p.E;
       RowTopK<KMAX> top;
       top.reset();
       const uint32_t acc_addr = lane_base + buf * p.acc_stride;
-      // 64 columns per round trip: two loads, one wait
-      for (int c0 = 0; c0 < ncols; c0 += 64) {
-        uint32_t r0[32], r1[32];
-        const bool second = c0 + 32 < ncols;  // warp-uniform
-        tmem_ld_32(acc_addr + c0, r0);
-        if (second) tmem_ld_32(acc_addr + c0 + 32, r1);
-        tmem_ld_wait();
-        offer_chunk(top, r0, c0, ncols, col_base);
-        if (second) offer_chunk(top, r1, c0 + 32, ncols, col_base);
+      // full tiles: one pass over columns [0, E); half tiles: one per chunk
+      const int passes = w.half ? p.n_chunks : 1;
+      for (int c = 0; c < passes; ++c) {
+        int col_base = 0, ncols = p.E;
+        uint32_t chunk_addr = acc_addr;
+        if (w.half) {
+          col_base = c * N_CHUNK + (upper ? chunk_n(p, c) / 2 : 0);
+          ncols = min(chunk_n(p, c) / 2, p.E - col_base);
+          chunk_addr += static_cast<uint32_t>(c * N_CHUNK);
+        }
+        // 64 columns per round trip: two loads, one wait
+        for (int c0 = 0; c0 < ncols; c0 += 64) {
+          uint32_t r0[32], r1[32];
+          const bool second = c0 + 32 < ncols;  // warp-uniform
+          tmem_ld_32(chunk_addr + c0, r0);
+          if (second) tmem_ld_32(chunk_addr + c0 + 32, r1);
+          tmem_ld_wait();
+          offer_chunk(top, r0, c0, ncols, col_base);
+          if (second) offer_chunk(top, r1, c0 + 32, ncols, col_base);
+        }
       }
       // the accumulator buffer may be overwritten once every epilogue warp of
       // the pair has read it

@@ -20,6 +20,11 @@
 //      row), keeps a top-k of the segment, and the G lists are merged with warp
 //      shuffles; then softmax and store.
 //
+// More than 256 experts (up to 512): one MMA per chunk of at most 256 experts
+// and K step (chunk c in tensor-memory columns from 256c), and steps 2..5 run
+// once per 256-expert column range: each pass pushes and reduces its columns
+// and the owners keep their running top-k lists across passes.
+//
 // Nothing but scores and ids is written to global memory.
 #pragma once
 
@@ -43,12 +48,14 @@ constexpr int PUSH_SCRATCH_BYTES = 32 * PUSH_SCRATCH_STRIDE * 4;   // one 32 x 3
 
 struct SplitHParams {
   int32_t T, H, E, k;
-  int32_t n_pad;        // MMA N (E rounded up to 16)
+  int32_t n_pad;        // total MMA N (E rounded up to 16, <= 512)
+  int32_t n_chunks;     // ceil(n_pad / 256): MMAs per K step, and exchange passes
+  int32_t kps;          // K slices per ring stage (2, or 1 when n_pad > 256)
   int32_t num_tiles;    // 128-token tiles
   int32_t k_blocks;     // ceil(H / 64)
   int32_t stages;
   int32_t b_boxes;
-  int32_t row_stride;   // floats per staged partial row (round_up(E, 32) + 4)
+  int32_t row_stride;   // floats per staged partial row (round_up(min(E, 256), 32) + 4)
   uint32_t tmem_cols;
   uint64_t timeout_ns;
   float* scores;
@@ -63,9 +70,9 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align_1024(smem_dyn);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + p.stages * KB_PER_STAGE * A_STAGE_BYTES;
+  uint8_t* sB = smem + p.stages * p.kps * A_STAGE_BYTES;
   float* staging = reinterpret_cast<float*>(smem);  // reuses the ring once every CTA's MMAs are done
-  float* scratch = reinterpret_cast<float*>(sB + p.stages * KB_PER_STAGE * p.b_boxes * B_BOX_BYTES);  // after the ring
+  float* scratch = reinterpret_cast<float*>(sB + p.stages * p.kps * p.b_boxes * B_BOX_BYTES);  // after the ring
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scratch) + PUSH_WARPS * PUSH_SCRATCH_BYTES);
   uint64_t* empty = full + p.stages;
   uint64_t* acc_full = empty + p.stages;
@@ -111,13 +118,13 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
       const uint32_t slice_tx = A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES;
       uint32_t stage = 0, phase = 0;
       int issued = 0;
-      for (int kb = kb0; kb < kb1; kb += KB_PER_STAGE) {
-        // a stage holds up to KB_PER_STAGE slices, never past this CTA's H slice
-        const int n_sub = min(KB_PER_STAGE, kb1 - kb);
+      for (int kb = kb0; kb < kb1; kb += p.kps) {
+        // a stage holds up to kps slices, never past this CTA's H slice
+        const int n_sub = min(p.kps, kb1 - kb);
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER, p.err_word)) break;
         mbar_arrive_expect_tx(&full[stage], n_sub * slice_tx);
         for (int sub = 0; sub < n_sub; ++sub) {
-          const int slot = stage * KB_PER_STAGE + sub;
+          const int slot = stage * p.kps + sub;
           const int k0 = (kb + sub) * BLOCK_K;
           tma_load_2d(sA + slot * A_STAGE_BYTES, &map_x, &full[stage], k0, tile * BLOCK_M, pol_x);
           for (int j = 0; j < p.b_boxes; ++j)
@@ -143,24 +150,38 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      const uint32_t idesc = idesc_bf16_f32(BLOCK_M, p.n_pad, false, true);
+      // chunk c: N = min(256, n_pad - 256c); its gate boxes start at box 4c
+      const uint32_t idesc0 = idesc_bf16_f32(BLOCK_M, min(p.n_pad, 256), false, true);
+      const uint32_t idesc1 = idesc_bf16_f32(BLOCK_M, p.n_pad > 256 ? p.n_pad - 256 : 256, false, true);
+      const bool two_chunks = p.n_chunks > 1;
       uint32_t stage = 0, phase = 0;
       bool ok = true;
-      for (int kb = kb0; kb < kb1; kb += KB_PER_STAGE) {
-        const int n_sub = min(KB_PER_STAGE, kb1 - kb);
+      for (int kb = kb0; kb < kb1; kb += p.kps) {
+        const int n_sub = min(p.kps, kb1 - kb);
         if (!mbar_wait(&full[stage], phase, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
         for (int sub = 0; sub < n_sub; ++sub) {
-          const int slot = stage * KB_PER_STAGE + sub;
+          const int slot = stage * p.kps + sub;
           const uint32_t a_addr = smem_u32(sA + slot * A_STAGE_BYTES);
           const uint32_t b_addr = smem_u32(sB + slot * p.b_boxes * B_BOX_BYTES);
+          if (two_chunks) {  // loop-invariant: no branch between the MMAs of a slice
 #pragma unroll
-          for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
-            umma_bf16(tmem_base, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc,
-                      (kb + sub != kb0) | kk);
+            for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
+              const uint32_t accumulate = (kb + sub != kb0) | kk;
+              const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
+              umma_bf16(tmem_base, a_desc, b_desc_k_slice(b_addr, kk), idesc0, accumulate);
+              umma_bf16(tmem_base + N_CHUNK, a_desc, b_desc_k_slice(b_addr + (N_CHUNK / B_BOX_N) * B_BOX_BYTES, kk),
+                        idesc1, accumulate);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
+              umma_bf16(tmem_base, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc0,
+                        (kb + sub != kb0) | kk);
+          }
         }
         umma_commit(&empty[stage]);
         if (++stage == static_cast<uint32_t>(p.stages)) {
@@ -183,110 +204,114 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     acc_ok = mbar_wait(acc_full, 0, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
     acc_ok = __all_sync(0xffffffffu, acc_ok);
   }
-  tc_fence_before_sync();
-  cluster_arrive_release();
-  cluster_wait_acquire();
-  tc_fence_after_sync();
 
-  // ---------------- push partial rows to their owners ----------------
-  // Each 32-row x 32-column chunk (row per thread from tensor memory) is
-  // transposed through this warp's scratch so that every remote store writes 128
-  // contiguous bytes of one row: 8 lanes per row, 4 rows per store instruction.
-  if (push_warp) {
-    const int quad = warp & 3;
-    if (acc_ok && quad * 32 < valid_rows) {
-      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-      float* my_scratch = scratch + (warp - 2) * (PUSH_SCRATCH_BYTES / 4);
-      const int sub_row = lane >> 3;       // 0..3: row within a group of 4
-      const int col4 = (lane & 7) * 4;     // column offset within the chunk
-      // 64 columns per tensor-memory round trip, pushed as two 32-column chunks
-      for (int c0 = 0; c0 < p.E; c0 += 64) {
-        uint32_t v[2][32];
-        const bool second = c0 + 32 < p.E;  // warp-uniform
-        tmem_ld_32(lane_base + c0, v[0]);
-        if (second) tmem_ld_32(lane_base + c0 + 32, v[1]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h == 1 && !second) break;
-          const int cc = c0 + 32 * h;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(my_scratch + lane * PUSH_SCRATCH_STRIDE + j) =
-                make_float4(__uint_as_float(v[h][j]), __uint_as_float(v[h][j + 1]), __uint_as_float(v[h][j + 2]),
-                            __uint_as_float(v[h][j + 3]));
-          __syncwarp();
-#pragma unroll
-          for (int rr = 0; rr < 32; rr += 4) {
-            const int t = quad * 32 + rr + sub_row;  // tile-local row
-            if (t < valid_rows && cc + col4 < p.E) {
-              const float4 val =
-                  *reinterpret_cast<const float4*>(my_scratch + (rr + sub_row) * PUSH_SCRATCH_STRIDE + col4);
-              float* dst = staging + static_cast<size_t>((t / C) * C + static_cast<int>(r)) * p.row_stride + cc + col4;
-              const unsigned owner = static_cast<unsigned>(t % C);
-              float* target = owner == r ? dst : static_cast<float*>(__cluster_map_shared_rank(dst, owner));
-              *reinterpret_cast<float4*>(target) = val;
-            }
-          }
-          __syncwarp();
-        }
-      }
-    }
-  }
-  tc_fence_before_sync();
-  cluster_arrive_release();  // every owner's staging area is complete past this point
-  cluster_wait_acquire();
-  if (warp == 1) {  // all tensor-memory reads of this CTA are done
+  // Owned rows: n_own <= 64 (C >= 2), and group * n_own <= SPLIT_THREADS, so one
+  // pass over the owned rows covers them all.
+  const int n_own = valid_rows > static_cast<int>(r) ? (valid_rows - static_cast<int>(r) + C - 1) / C : 0;
+  int group = 32;  // threads per owned row: a power of two
+  while (group > 1 && (n_own * group > SPLIT_THREADS || group * 8 > min(p.E, N_CHUNK))) group >>= 1;
+  const int slot = static_cast<int>(threadIdx.x) / group;
+  const int seg = threadIdx.x % group;
+  const bool active = slot < n_own;
+  RowTopK<KMAX> top;
+  top.reset();
+
+  for (int pass = 0; pass < p.n_chunks; ++pass) {
+    const int col0 = pass * N_CHUNK;                   // first expert of this pass
+    const int pass_cols = min(N_CHUNK, p.E - col0);
+    // every ring (first pass) or every staging area (later passes) is free
+    tc_fence_before_sync();
+    cluster_arrive_release();
+    cluster_wait_acquire();
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, p.tmem_cols);
-  }
 
-  // ---------------- reduce owned rows, top-k, softmax ----------------
-  {
-    const int n_own = valid_rows > static_cast<int>(r) ? (valid_rows - static_cast<int>(r) + C - 1) / C : 0;
-    int group = 32;  // threads per owned row: a power of two
-    while (group > 1 && (n_own * group > SPLIT_THREADS || group * 8 > p.E)) group >>= 1;
-    const int rows_per_pass = SPLIT_THREADS / group;
-    const int passes = (n_own + rows_per_pass - 1) / rows_per_pass;
-    const int seg = threadIdx.x % group;
-    for (int pass = 0; pass < passes; ++pass) {
-      const int slot = pass * rows_per_pass + static_cast<int>(threadIdx.x) / group;
-      const bool active = slot < n_own;
-      RowTopK<KMAX> top;
-      top.reset();
-      if (active) {
-        // segment `seg` takes every group-th float4 of the row: consecutive lanes
-        // read consecutive 16-byte words (no bank conflicts), and each thread still
-        // offers its columns in increasing order
-        const float* rows = staging + static_cast<size_t>(slot) * C * p.row_stride;
-        const int c_end = p.E;
-        for (int c = 4 * seg; c < c_end; c += 4 * group) {
-          float4 v[C];
+    // ---------------- push partial rows to their owners ----------------
+    // Each 32-row x 32-column chunk (row per thread from tensor memory) is
+    // transposed through this warp's scratch so that every remote store writes 128
+    // contiguous bytes of one row: 8 lanes per row, 4 rows per store instruction.
+    if (push_warp) {
+      const int quad = warp & 3;
+      if (acc_ok && quad * 32 < valid_rows) {
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
+        float* my_scratch = scratch + (warp - 2) * (PUSH_SCRATCH_BYTES / 4);
+        const int sub_row = lane >> 3;       // 0..3: row within a group of 4
+        const int col4 = (lane & 7) * 4;     // column offset within the chunk
+        // 64 columns per tensor-memory round trip, pushed as two 32-column chunks
+        for (int c0 = 0; c0 < pass_cols; c0 += 64) {
+          uint32_t v[2][32];
+          const bool second = c0 + 32 < pass_cols;  // warp-uniform
+          tmem_ld_32(lane_base + c0, v[0]);
+          if (second) tmem_ld_32(lane_base + c0 + 32, v[1]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < C; ++q) v[q] = *reinterpret_cast<const float4*>(rows + q * p.row_stride + c);
-          float4 acc = v[0];
+          for (int h = 0; h < 2; ++h) {
+            if (h == 1 && !second) break;
+            const int cc = c0 + 32 * h;
 #pragma unroll
-          for (int q = 1; q < C; ++q) {  // rank order: the same sum whichever CTA owns the row
-            acc.x += v[q].x;
-            acc.y += v[q].y;
-            acc.z += v[q].z;
-            acc.w += v[q].w;
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(my_scratch + lane * PUSH_SCRATCH_STRIDE + j) =
+                  make_float4(__uint_as_float(v[h][j]), __uint_as_float(v[h][j + 1]), __uint_as_float(v[h][j + 2]),
+                              __uint_as_float(v[h][j + 3]));
+            __syncwarp();
+#pragma unroll
+            for (int rr = 0; rr < 32; rr += 4) {
+              const int t = quad * 32 + rr + sub_row;  // tile-local row
+              if (t < valid_rows && cc + col4 < pass_cols) {
+                const float4 val =
+                    *reinterpret_cast<const float4*>(my_scratch + (rr + sub_row) * PUSH_SCRATCH_STRIDE + col4);
+                float* dst =
+                    staging + static_cast<size_t>((t / C) * C + static_cast<int>(r)) * p.row_stride + cc + col4;
+                const unsigned owner = static_cast<unsigned>(t % C);
+                float* target = owner == r ? dst : static_cast<float*>(__cluster_map_shared_rank(dst, owner));
+                *reinterpret_cast<float4*>(target) = val;
+              }
+            }
+            __syncwarp();
           }
-          top.offer(acc.x, c);
-          if (c + 1 < c_end) top.offer(acc.y, c + 1);
-          if (c + 2 < c_end) top.offer(acc.z, c + 2);
-          if (c + 3 < c_end) top.offer(acc.w, c + 3);
         }
       }
-      merge_lane_groups(top, group);
-      if (active && seg == 0) {
-        const int t_local = static_cast<int>(r) + C * slot;
-        const int64_t row = static_cast<int64_t>(tile) * BLOCK_M + t_local;
-        top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+    }
+    tc_fence_before_sync();
+    cluster_arrive_release();  // every owner's staging area is complete past this point
+    cluster_wait_acquire();
+    if (warp == 1 && pass + 1 == p.n_chunks) {  // all tensor-memory reads of this CTA are done
+      tc_fence_after_sync();
+      tmem_dealloc(tmem_base, p.tmem_cols);
+    }
+
+    // ---------------- reduce owned rows of this pass into the running top-k ----------------
+    if (active) {
+      // segment `seg` takes every group-th float4 of the row: consecutive lanes
+      // read consecutive 16-byte words (no bank conflicts), and each thread still
+      // offers its columns in increasing order
+      const float* rows = staging + static_cast<size_t>(slot) * C * p.row_stride;
+      for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
+        float4 v[C];
+#pragma unroll
+        for (int q = 0; q < C; ++q) v[q] = *reinterpret_cast<const float4*>(rows + q * p.row_stride + c);
+        float4 acc = v[0];
+#pragma unroll
+        for (int q = 1; q < C; ++q) {  // rank order: the same sum whichever CTA owns the row
+          acc.x += v[q].x;
+          acc.y += v[q].y;
+          acc.z += v[q].z;
+          acc.w += v[q].w;
+        }
+        top.offer(acc.x, col0 + c);
+        if (c + 1 < pass_cols) top.offer(acc.y, col0 + c + 1);
+        if (c + 2 < pass_cols) top.offer(acc.z, col0 + c + 2);
+        if (c + 3 < pass_cols) top.offer(acc.w, col0 + c + 3);
       }
     }
   }
 
+  // ---------------- merge the segments, softmax, store ----------------
+  merge_lane_groups(top, group);
+  if (active && seg == 0) {
+    const int t_local = static_cast<int>(r) + C * slot;
+    const int64_t row = static_cast<int64_t>(tile) * BLOCK_M + t_local;
+    top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+  }
 }
 
 }  // namespace tkg

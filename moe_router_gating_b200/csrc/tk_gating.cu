@@ -40,20 +40,24 @@ tk_status validate_sizes(int64_t T, int64_t H, int64_t E, int32_t k) {
   return TK_OK;
 }
 
+// Floats per staged partial row of the split-H exchange (one pass of up to 256
+// experts; +4 spreads the rows over the shared-memory banks).
+int split_row_stride(int64_t E) { return round_up(static_cast<int>(E < tkg::N_CHUNK ? E : tkg::N_CHUNK), 32) + 4; }
+
 constexpr int kMaxSplit = 16;  // CTAs per cluster in the split-H variant (16 needs non-portable clusters)
 
 // Split-H plan: one 128-token tile per cluster of C CTAs, single-CTA MMAs.
 tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* plan) {
   const int n_pad = round_up(static_cast<int>(E), 16);
+  const int kps = n_pad > tkg::N_CHUNK ? 1 : tkg::KB_PER_STAGE;  // a slice of 512 experts is 80 KB
   const int b_boxes = (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES;
   const int scratch = tkg::PUSH_WARPS * tkg::PUSH_SCRATCH_BYTES;
-  int stages = (kMaxDynamicSmem - kSmemReserve - scratch) / (tkg::KB_PER_STAGE * stage_bytes);
+  int stages = (kMaxDynamicSmem - kSmemReserve - scratch) / (kps * stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
-  const int row_stride = round_up(static_cast<int>(E), 32) + 4;
-  // the staged partial rows of a tile reuse the ring
-  if (stages < 2 || tkg::BLOCK_M * row_stride * 4 > stages * tkg::KB_PER_STAGE * stage_bytes)
-    return TK_ERR_UNSUPPORTED;
+  const int row_stride = split_row_stride(E);
+  // the staged partial rows of a tile (one 256-expert pass at a time) reuse the ring
+  if (stages < 2 || tkg::BLOCK_M * row_stride * 4 > stages * kps * stage_bytes) return TK_ERR_UNSUPPORTED;
   const int64_t tiles = (T + tkg::BLOCK_M - 1) / tkg::BLOCK_M;
   plan->variant = TK_VARIANT_SPLIT_H;
   plan->block_m = tkg::BLOCK_M;
@@ -65,8 +69,9 @@ tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* p
   plan->grid = static_cast<int32_t>(tiles * C);
   plan->cluster = C;
   plan->threads = tkg::SPLIT_THREADS;
-  plan->smem_bytes = stages * tkg::KB_PER_STAGE * stage_bytes + scratch + kSmemReserve;
+  plan->smem_bytes = stages * kps * stage_bytes + scratch + kSmemReserve;
   plan->tmem_cols = static_cast<int32_t>(pow2_at_least(round_up(n_pad, 32)));
+  plan->slices_per_stage = kps;
   return TK_OK;
 }
 
@@ -117,6 +122,7 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   const int cg = pair ? 2 : 1;
   const int n_pad = pair ? round_up(static_cast<int>(E), 128) : round_up(static_cast<int>(E), 16);
   const int acc_stride = round_up(n_pad, 32);
+  const int acc_bufs = 2 * acc_stride <= 512 ? 2 : 1;  // 512 tensor-memory columns
   const int b_boxes = pair ? n_pad / 2 / tkg::B_BOX_N : (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::KB_PER_STAGE * (tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES);
   int stages = (kMaxDynamicSmem - kSmemReserve) / stage_bytes;
@@ -152,7 +158,8 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   plan->cluster = cg;
   plan->threads = tkg::ROW_TILE_THREADS;
   plan->smem_bytes = stages * stage_bytes + kSmemReserve;
-  plan->tmem_cols = static_cast<int32_t>(pow2_at_least(2 * acc_stride));
+  plan->tmem_cols = static_cast<int32_t>(pow2_at_least(acc_bufs * acc_stride));
+  plan->slices_per_stage = tkg::KB_PER_STAGE;
   return TK_OK;
 }
 
@@ -271,7 +278,7 @@ const DeviceState* device_state() {
   }
   void* err = nullptr;
   if (cudaGetSymbolAddress(&err, g_tk_error_word) != cudaSuccess || !set_up_kernels<1>() || !set_up_kernels<2>() ||
-      !set_up_kernels<4>() || !set_up_kernels<8>() || !set_up_kernels<16>()) {
+      !set_up_kernels<4>() || !set_up_kernels<8>() || !set_up_kernels<16>() || !set_up_kernels<32>()) {
     cudaGetLastError();
     return nullptr;  // not cached: a later call retries
   }
@@ -380,11 +387,13 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
     sp.E = static_cast<int32_t>(E);
     sp.k = k;
     sp.n_pad = pl.n_pad;
+    sp.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
+    sp.kps = pl.slices_per_stage;
     sp.num_tiles = pl.num_tiles;
     sp.k_blocks = pl.k_blocks;
     sp.stages = pl.stages;
     sp.b_boxes = (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
-    sp.row_stride = round_up(static_cast<int>(E), 32) + 4;
+    sp.row_stride = split_row_stride(E);
     sp.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
     sp.timeout_ns = g_timeout_ns;
     sp.scores = scores;
@@ -394,7 +403,8 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
     if (k <= 2) return launch_split_h<2>(pl, dev->max_split_cluster, mx, mw, sp, stream);
     if (k <= 4) return launch_split_h<4>(pl, dev->max_split_cluster, mx, mw, sp, stream);
     if (k <= 8) return launch_split_h<8>(pl, dev->max_split_cluster, mx, mw, sp, stream);
-    return launch_split_h<16>(pl, dev->max_split_cluster, mx, mw, sp, stream);
+    if (k <= 16) return launch_split_h<16>(pl, dev->max_split_cluster, mx, mw, sp, stream);
+    return launch_split_h<32>(pl, dev->max_split_cluster, mx, mw, sp, stream);
   }
 
   tkg::RowTileParams prm;
@@ -403,7 +413,9 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   prm.E = static_cast<int32_t>(E);
   prm.k = k;
   prm.n_pad = pl.n_pad;
+  prm.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
   prm.acc_stride = round_up(pl.n_pad, 32);
+  prm.acc_bufs = 2 * prm.acc_stride <= 512 ? 2 : 1;
   prm.num_tiles = pl.num_tiles;
   prm.num_half = pl.num_half_tiles;
   prm.k_blocks = pl.k_blocks;
@@ -420,7 +432,8 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   if (k <= 2) return launch_row_variant<2>(pl, mx, mx64, mw, prm, stream);
   if (k <= 4) return launch_row_variant<4>(pl, mx, mx64, mw, prm, stream);
   if (k <= 8) return launch_row_variant<8>(pl, mx, mx64, mw, prm, stream);
-  return launch_row_variant<16>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 16) return launch_row_variant<16>(pl, mx, mx64, mw, prm, stream);
+  return launch_row_variant<32>(pl, mx, mx64, mw, prm, stream);
 }
 
 }  // namespace

@@ -45,8 +45,8 @@ def test_status_strings():
     ((8, 60, 16, 2), tk.TK_ERR_UNSUPPORTED),        # H % 8
     ((8, 64, 20, 2), tk.TK_ERR_UNSUPPORTED),        # E % 8
     ((8, 64, 8, 2), tk.TK_ERR_UNSUPPORTED),         # E < 16
-    ((8, 64, 264, 2), tk.TK_ERR_UNSUPPORTED),       # E > 256
-    ((8, 64, 64, 17), tk.TK_ERR_UNSUPPORTED),       # k > 16
+    ((8, 64, 520, 2), tk.TK_ERR_UNSUPPORTED),       # E > 512
+    ((8, 64, 64, 33), tk.TK_ERR_UNSUPPORTED),       # k > 32
 ])
 def test_invalid_sizes_rejected_before_cuda(args, code):
     T, H, E, k = args
@@ -87,7 +87,7 @@ def test_plans_for_router_workloads():
         if p["variant"] == 1:
             assert p["grid"] == min(p["num_tiles"], 148) and p["cluster"] == 1
         if p["variant"] == 3:
-            assert p["cluster"] == 2 and p["block_m"] == 256 and p["n_pad"] in (128, 256)
+            assert p["cluster"] == 2 and p["block_m"] == 256 and p["n_pad"] in (128, 256, 384, 512)
             assert p["grid"] == 2 * min(p["num_tiles"], 74)
         if p["variant"] == 2:
             C = p["cluster"]
@@ -123,9 +123,28 @@ def test_plan_variant_choice():
 
 def test_plan_tmem_and_smem_budget():
     for T in (1, 1000, 30000):
-        for E in range(16, 257, 8):
+        for E in range(16, 513, 8):
             p = tk.make_plan(T, 7168, E, min(8, E), 148)
-            buffers = 1 if p["variant"] == 2 else 2  # split-H keeps one accumulator
-            assert p["tmem_cols"] >= buffers * ((p["n_pad"] + 31) // 32 * 32)
+            acc = (p["n_pad"] + 31) // 32 * 32
+            # split-H keeps one accumulator; row tiles two, or one when two do not fit
+            buffers = 1 if p["variant"] == 2 or 2 * acc > 512 else 2
+            assert p["tmem_cols"] >= buffers * acc
             assert p["tmem_cols"] <= 512
             assert p["smem_bytes"] <= 232448
+            assert p["stages"] >= 2 and p["slices_per_stage"] in (1, 2)
+            if p["variant"] == 2:
+                # the exchange stages 128 rows of up to 256 experts in the ring
+                ring = p["smem_bytes"] - 4 * 32 * 36 * 4 - 1280
+                row_stride = (min(E, 256) + 31) // 32 * 32 + 4
+                assert 128 * row_stride * 4 <= ring
+
+
+def test_plan_large_expert_counts():
+    p = tk.make_plan(65536, 7168, 512, 8, 148)      # pairs, two 256-expert MMA chunks, one accumulator
+    assert p["variant"] == 3 and p["n_pad"] == 512 and p["tmem_cols"] == 512
+    p = tk.make_plan(65536, 7168, 320, 8, 148)      # 384 columns: chunks of 256 and 128
+    assert p["variant"] == 3 and p["n_pad"] == 384 and p["tmem_cols"] == 512
+    p = tk.make_plan(4096, 7168, 512, 32, 148)      # split-H, one 80 KB K slice per stage
+    assert p["variant"] == 2 and p["slices_per_stage"] == 1 and p["tmem_cols"] == 512
+    p = tk.make_plan(4096, 7168, 256, 8, 148)
+    assert p["slices_per_stage"] == 2

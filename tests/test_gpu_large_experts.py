@@ -1,0 +1,74 @@
+"""Parity on the GPU for more than 256 experts (two MMA chunks of at most 256
+experts each) and for up to 32 selected experts, against the CPU oracle under
+the rule of tests/parity.py.  Covers both kernel families (split-H clusters
+for few tokens, CTA pairs with a single-buffered accumulator for many), pair
+half tiles, E padding inside the second chunk, and exact ties across the
+chunk boundary and across the halves a pair's CTAs hold."""
+import numpy as np
+import pytest
+import torch
+
+import moe_router_gating_b200 as tk
+import oracle
+import parity
+import workloads
+from gpu_helpers import check_against_oracle, check_workload, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def clean_error_word():
+    assert torch.cuda.is_available()
+    tk.device_error(clear=True)
+    yield
+    assert tk.device_error(clear=True) == 0, "a kernel wait expired during the GPU tests"
+
+
+@pytest.mark.parametrize("T,H,E,k", [
+    # split-H clusters
+    (1, 7168, 512, 8), (7, 1024, 512, 32), (128, 2048, 320, 16), (1000, 1024, 512, 32), (4096, 1024, 384, 8),
+    (129, 512, 264, 1), (300, 520, 504, 17),
+    # CTA pairs, two chunks, single accumulator (and half tiles: T just above a full round)
+    (20000, 512, 512, 8), (30000, 512, 320, 32), (19999, 256, 448, 5), (40000, 128, 264, 3),
+    # k up to 32 with one chunk
+    (2000, 1024, 256, 32), (40000, 512, 256, 32), (5000, 256, 64, 32), (700, 256, 32, 32),
+])
+def test_large_expert_shapes(T, H, E, k):
+    check_workload(workloads.RouterWorkload(f"large_{T}_{H}_{E}_{k}", T, H, E, k, seed=5))
+
+
+@pytest.mark.parametrize("T", [300, 24000])
+def test_ties_across_chunk_and_half_boundaries(T):
+    # equal gate columns give equal logits: the lower expert index must win,
+    # whichever chunk, pair half or CTA holds the other copy
+    E, H, k = 512, 512, 8
+    wl = workloads.RouterWorkload(f"ties_{T}", T, H, E, k, seed=13)
+    w = wl.gate_weight().copy()
+    pairs = ((255, 256), (127, 128), (383, 384), (0, 511), (300, 301), (64, 448))
+    for a, b in pairs:
+        w[:, b] = w[:, a]
+    # make the tied columns competitive: scale them up
+    for a, b in pairs:
+        w[:, a] = workloads.round_bf16(workloads.bf16_to_f64(w[:, a]) * 3.0)
+        w[:, b] = w[:, a]
+    check_against_oracle(wl.hidden(), w, k, duplicate_pairs=pairs, label=f"ties_{T}")
+
+
+def test_large_e_workload_sampled_rows():
+    """The 65536 x 7168 x 512 launch the benchmark times; the oracle checks sampled rows."""
+    wl = workloads.LARGE_E
+    x_bits = wl.hidden()
+    w_bits = wl.gate_weight()
+    s, i = run_gpu(x_bits, w_bits, wl.k)
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([np.arange(0, 256), np.arange(wl.T - 256, wl.T),
+                                     rng.choice(wl.T, 512, replace=False)]))
+    ref = oracle.fused_topk_gating(x_bits[rows], w_bits, wl.k, want_logits=True)
+    parity.check(s, i, ref, rows=rows, label="large_e-sampled")
+    assert np.all((i >= 0) & (i < wl.E))
+    assert np.all(np.diff(s, axis=1) <= 0)
+
+
+def test_large_k_workload():
+    check_workload(workloads.LARGE_K)

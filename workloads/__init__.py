@@ -171,7 +171,12 @@ TRAIN = RouterWorkload("train", 65536, 7168, 256, 8)
 DECODE_TS = (1, 8, 32, 128, 256)
 DECODE = tuple(RouterWorkload(f"decode_T{t}", t, 7168, 256, 8) for t in DECODE_TS)
 
-WORKLOADS = {w.name: w for w in (TINY, DEEPSEEK, SKEW, TRAIN) + DECODE}
+# More experts and larger k than the pages' router (fine-grained MoE): two MMA
+# chunks of 256 experts, top-32 selection.
+LARGE_E = RouterWorkload("large_e", 65536, 7168, 512, 8)
+LARGE_K = RouterWorkload("large_k", 4096, 7168, 512, 32)
+
+WORKLOADS = {w.name: w for w in (TINY, DEEPSEEK, SKEW, TRAIN, LARGE_E, LARGE_K) + DECODE}
 
 
 def expert_ids(T: int, k: int, E: int, seed: int, kind: str = "uniform") -> np.ndarray:
