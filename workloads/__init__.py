@@ -179,6 +179,28 @@ LARGE_K = RouterWorkload("large_k", 4096, 7168, 512, 32)
 WORKLOADS = {w.name: w for w in (TINY, DEEPSEEK, SKEW, TRAIN, LARGE_E, LARGE_K) + DECODE}
 
 
+def quantize_e4m3_rows(values: np.ndarray):
+    """Per-row FP8 E4M3 quantization of a float array [R, C]: scale = max|row| / 448
+    (1 for an all-zero row), bits = e4m3(row / scale) rounded to nearest even by
+    torch's float8_e4m3fn cast.  Returns (uint8 bits [R, C], float32 scales [R]).
+    Input preparation only (the pages' per-token quantize); no gating arithmetic."""
+    import torch
+    v = torch.from_numpy(np.ascontiguousarray(values, dtype=np.float32))
+    amax = v.abs().amax(dim=1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    q = (v / scale[:, None]).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8).numpy().copy(), scale.numpy().astype(np.float32)
+
+
+def fp8_inputs(wl: "RouterWorkload"):
+    """FP8 versions of a workload's inputs: the bf16 hidden rows quantized per token,
+    the bf16 gate quantized per expert and stored expert-major [E, H].
+    Returns (hidden_q [T, H], hidden_scale [T], gate_q [E, H], gate_scale [E])."""
+    xq, xs = quantize_e4m3_rows(bf16_to_f64(wl.hidden()).astype(np.float32))
+    wq, ws = quantize_e4m3_rows(bf16_to_f64(wl.gate_weight()).T.astype(np.float32))
+    return xq, xs, wq, ws
+
+
 def expert_ids(T: int, k: int, E: int, seed: int, kind: str = "uniform") -> np.ndarray:
     """Seeded int32 ``[T, k]`` expert ids, k distinct per row (as a router emits).
 
