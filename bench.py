@@ -7,7 +7,8 @@ router, T=65536 tokens, H=7168, E=256 experts, k=8 (hidden 940 MB > L2).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-``--op route`` times the routing metadata (per-expert offsets, the expert-grouped
+``--precision fp8`` times the FP8 (E4M3) entry point on the workload's inputs
+quantized per token (hidden) and per expert (gate).  ``--op route`` times the routing metadata (per-expert offsets, the expert-grouped
 order and each assignment's position) of seeded ids of the workload's T x k
 shape; ``--op gating_route`` times gating followed by routing of its ids.
 
@@ -59,6 +60,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (profiling cases)")
+    ap.add_argument("--precision", default="bf16", choices=("bf16", "fp8"),
+                    help="bf16 (default) or FP8 E4M3 inputs with per-token / per-expert scales")
     ap.add_argument("--op", default="gating", choices=("gating", "route", "gating_route"),
                     help="gating (default); route: routing metadata of the workload's T x k ids; "
                          "gating_route: both, chained on the device")
@@ -220,10 +223,10 @@ def kernel_source_digest() -> str:
     return tkbuild.gating_kernel_digest()
 
 
-def profiled_traffic(wl, digest: str):
+def profiled_traffic(wl, digest: str, suffix: str = ""):
     """dram read+write bytes per launch from a committed ncu summary, if it was
     taken on the current kernel sources (same digest); else None."""
-    path = os.path.join(PROFILE_DIR, f"traffic_{wl.name}.txt")
+    path = os.path.join(PROFILE_DIR, f"traffic_{wl.name}{suffix}.txt")
     if not os.path.exists(path):
         return None, None
     vals = {}
@@ -283,20 +286,30 @@ def run_ours(args, wl):
 
     # ---- inputs: seeded host arrays, each rank gates its own token shard ----
     rank_wl = rank_workload(wl, rank)
-    x_bits = rank_wl.hidden()
-    w_bits = rank_wl.gate_weight()
-    x_host = workloads.to_torch_bf16(x_bits)
-    w = workloads.to_torch_bf16(w_bits).to(dev)
-    hidden_bytes = wl.T * wl.H * 2
-    big = hidden_bytes > L2_BYTES
-    x = x_host.to(dev)
+    fp8 = args.precision == "fp8"
     scores = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
     ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
-    flush = None if big else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if fp8:
+        xq, xs, wq, ws = workloads.fp8_inputs(rank_wl)
+        x_host = torch.from_numpy(xq)
+        xs_host = torch.from_numpy(xs)
+        x, xsd = x_host.to(dev), xs_host.to(dev)
+        wqd, wsd = torch.from_numpy(wq).to(dev), torch.from_numpy(ws).to(dev)
+        hidden_bytes = wl.T * wl.H + 4 * wl.T
 
-    def step():
-        tk.fused_topk_gating(x, w, wl.k, scores=scores, ids=ids, stream=stream)
+        def step():
+            tk.fused_topk_gating_fp8(x, xsd, wqd, wsd, wl.k, scores=scores, ids=ids, stream=stream)
+    else:
+        x_host = workloads.to_torch_bf16(rank_wl.hidden())
+        w = workloads.to_torch_bf16(rank_wl.gate_weight()).to(dev)
+        x = x_host.to(dev)
+        hidden_bytes = wl.T * wl.H * 2
+
+        def step():
+            tk.fused_topk_gating(x, w, wl.k, scores=scores, ids=ids, stream=stream)
+    big = hidden_bytes > L2_BYTES
+    flush = None if big else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -345,15 +358,27 @@ def run_ours(args, wl):
     s_host = torch.empty((wl.T, wl.k), dtype=torch.float32).pin_memory()
     i_host = torch.empty((wl.T, wl.k), dtype=torch.int32).pin_memory()
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    if fp8:
+        xs_pinned = xs_host.pin_memory()
+
+        def e2e_step():  # host buffers in and out around the public FP8 call
+            x.copy_(x_pinned, non_blocking=True)
+            xsd.copy_(xs_pinned, non_blocking=True)
+            tk.fused_topk_gating_fp8(x, xsd, wqd, wsd, wl.k, scores=scores, ids=ids, stream=stream)
+            s_host.copy_(scores, non_blocking=True)
+            i_host.copy_(ids, non_blocking=True)
+    else:
+        def e2e_step():
+            tk.fused_topk_gating_host(x_pinned, w, wl.k, s_host, i_host, x, scores, ids, stream=stream)
     for _ in range(2):
-        tk.fused_topk_gating_host(x_pinned, w, wl.k, s_host, i_host, x, scores, ids, stream=stream)
+        e2e_step()
     torch.cuda.synchronize(dev)
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        tk.fused_topk_gating_host(x_pinned, w, wl.k, s_host, i_host, x, scores, ids, stream=stream)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -368,17 +393,21 @@ def run_ours(args, wl):
     peaks, peak_src = load_peaks()
     bytes_alg = wl.algorithmic_bytes()
     flops = wl.flops()
+    tc_factor = 1.0
+    if fp8:  # 1-byte operands plus the scales; the FP8 tensor peak is twice the bf16 one (nominal ratio)
+        bytes_alg = wl.T * wl.H + wl.E * wl.H + 4 * (wl.T + wl.E) + 8 * wl.T * wl.k
+        tc_factor = 2.0
     t_s = launch_ms / 1e3
     hbm_ach = bytes_alg / t_s / 1e9
     tc_ach = flops / t_s / 1e12
     # a long run of back-to-back launches settles at the power-capped clock: the
     # tensor term then uses the sustained bf16 figure, a short one the burst figure
     sustained = elapsed_max_ms > 100.0 and "bf16_tflops_sustained" in peaks
-    tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    tc_peak = tc_factor * (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
     t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (tc_peak * 1e12)
     digest = kernel_source_digest()
-    traffic, traffic_src = profiled_traffic(wl, digest)
+    traffic, traffic_src = profiled_traffic(wl, digest, "_fp8" if fp8 else "")
     hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
            "frac": hbm_ach / peaks["hbm_gbs"], "traffic": traffic}
     tc = {"bound": "tensor", "achieved": tc_ach, "peak": tc_peak, "unit": "TFLOP/s",
@@ -387,7 +416,8 @@ def run_ours(args, wl):
     roofline = dict(primary)
     roofline.update({
         "peak_source": (f"{peak_src}; HBM = copy GB/s (of measured); tensor = cuBLAS bf16 "
-                        f"{'sustained (timed region > 100 ms)' if sustained else 'burst'} TFLOP/s (of measured)"),
+                        f"{'sustained (timed region > 100 ms)' if sustained else 'burst'} TFLOP/s (of measured)"
+                        + ("; x2 for FP8 (nominal FP8/bf16 ratio)" if fp8 else "")),
         "roofline_frac": max(t_hbm, t_tc) / t_s,
         "algorithmic_bytes_per_launch": bytes_alg, "flops_per_launch": flops,
         "launch_ms": launch_ms, "traffic_source": traffic_src,
@@ -395,10 +425,11 @@ def run_ours(args, wl):
         "secondary": {k: secondary[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
     })
 
-    plan = tk.make_plan(wl.T, wl.H, wl.E, wl.k, torch.cuda.get_device_properties(dev).multi_processor_count)
+    plan = tk.make_plan(wl.T, wl.H // 2 if fp8 else wl.H, wl.E, wl.k,
+                        torch.cuda.get_device_properties(dev).multi_processor_count)
 
     cpu = None
-    if not args.no_cpu_baseline and world == 1:
+    if not args.no_cpu_baseline and world == 1 and not fp8:
         v, rows, dt, cores = time_oracle(wl, args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"first {rows} of {wl.T} tokens ({dt:.1f} s, fp64 oracle with full sort, all host threads)"}
@@ -406,11 +437,14 @@ def run_ours(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
         "config": {
             "workload": workload_desc(wl), "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
             "tokens_per_rank_per_step": wl.T,
-            "arithmetic": "bf16 x bf16 products, fp32 accumulate (tcgen05), fp32 top-k and softmax",
+            "arithmetic": ("e4m3 x e4m3 products, fp32 accumulate (tcgen05 kind::f8f6f4), per-expert and per-token "
+                           "scales in fp32, fp32 top-k and softmax" if fp8 else
+                           "bf16 x bf16 products, fp32 accumulate (tcgen05), fp32 top-k and softmax"),
+            "precision": args.precision,
             "l2": ("inputs larger than L2: hidden is %.0f MB per step (gate %.2f MB stays L2-resident by design)"
                    % (hidden_bytes / 1e6, wl.H * wl.E * 2 / 1e6)) if big else
                   "L2 flushed (256 MB write) before every timed launch; each launch timed alone",
@@ -421,7 +455,9 @@ def run_ours(args, wl):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": hidden_bytes,
                 "d2h_bytes_per_step": wl.T * wl.k * 8,
-                "path": "tk_gating_fused_topk_host: pinned host hidden -> device, kernel, scores+ids -> pinned host"},
+                "path": ("pinned host hidden_q + scales -> device, tk_gating_fused_topk_fp8, scores+ids -> pinned host"
+                         if fp8 else
+                         "tk_gating_fused_topk_host: pinned host hidden -> device, kernel, scores+ids -> pinned host")},
         "gpu_launches": args.steps,
         "clocks": sampler.summary(),
     }

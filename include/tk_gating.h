@@ -108,6 +108,39 @@ TK_API tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* 
                                     int64_t E, int32_t k, float* scores_host, int32_t* ids_host, void* hidden_dev,
                                     float* scores_dev, int32_t* ids_dev, void* stream);
 
+/*
+ * tk_gating_fused_topk_fp8 -- the fused gating operator on FP8 (E4M3) inputs.
+ *
+ * The gating of section 4.1 on inputs quantized as the page's section 4.3
+ * "Quantization" describes (FP8 E4M3 values with a per-token scale, its
+ * per_token_quantize).  A tensor-core FP8 product needs both operands in FP8,
+ * so the gate is quantized too, with one scale per expert:
+ *
+ *   hidden[t, h] = hidden_scale[t] * e4m3(hidden_q[t, h])
+ *   gate[h, e]   = gate_scale[e]   * e4m3(gate_q[e, h])
+ *   logits[t, e] = (sum_h e4m3(hidden_q[t, h]) * e4m3(gate_q[e, h])) * gate_scale[e] * hidden_scale[t]
+ *
+ * The products are exact and summed in fp32 on the tensor cores
+ * (tcgen05.mma kind::f8f6f4); the two scales are applied in fp32 in that
+ * order; ranking, top-k and softmax as tk_gating_fused_topk.
+ *
+ *   hidden_q      device, E4M3 bytes [T, H] row-major.
+ *   hidden_scale  device, fp32 [T].
+ *   gate_q        device, E4M3 bytes [E, H] row-major: expert-major, each
+ *                 expert's H values contiguous (the layout of a quantized
+ *                 [E, H] linear weight with one scale per row).
+ *   gate_scale    device, fp32 [E].
+ *   T, E, k, scores, ids, stream  as tk_gating_fused_topk;  H % 16 == 0.
+ *
+ * Errors as tk_gating_fused_topk (every pointer, the scales included, must be
+ * 16-byte aligned; H not a multiple of 16 is TK_ERR_UNSUPPORTED).  The launch is
+ * the one tk_gating_make_plan gives for (T, H / 2, E, k): a K slice of 128 FP8
+ * values takes the shared memory of 64 bf16 values.
+ */
+TK_API tk_status tk_gating_fused_topk_fp8(const void* hidden_q, const float* hidden_scale, const void* gate_q,
+                                          const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k,
+                                          float* scores, int32_t* ids, void* stream);
+
 /* Kernel variants chosen by the planner. */
 typedef enum {
   TK_VARIANT_NONE = 0,        /* T == 0: nothing to launch */

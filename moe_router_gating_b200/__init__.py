@@ -23,6 +23,8 @@ from ._binding import (  # noqa: F401
     device_error,
     exported_symbols,
     fused_topk_gating,
+    fused_topk_gating_fp8,
+    fused_topk_gating_fp8_ptr,
     fused_topk_gating_host,
     fused_topk_gating_ptr,
     library,
@@ -37,7 +39,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "fused_topk_gating", "fused_topk_gating_host", "fused_topk_gating_ptr", "make_plan", "route", "route_plan",
+    "fused_topk_gating", "fused_topk_gating_fp8", "fused_topk_gating_host", "fused_topk_gating_ptr", "make_plan", "route", "route_plan",
     "route_ptr", "device_error",
     "set_wait_timeout_ns", "status_string", "TkGatingError", "library", "library_path",
 ]

@@ -58,6 +58,8 @@ def library() -> ctypes.CDLL:
             lib.tk_gating_fused_topk.restype = ctypes.c_int
             lib.tk_gating_fused_topk_host.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp]
             lib.tk_gating_fused_topk_host.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_fp8.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp]
+            lib.tk_gating_fused_topk_fp8.restype = ctypes.c_int
             lib.tk_gating_make_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(_Plan)]
             lib.tk_gating_make_plan.restype = ctypes.c_int
             lib.tk_gating_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -137,6 +139,45 @@ def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, st
         with torch.cuda.device(hidden.device):
             st = lib.tk_gating_fused_topk(*args, _stream_handle(stream, hidden.device))
     _check(st, "tk_gating_fused_topk")
+    return scores, ids
+
+
+def fused_topk_gating_fp8_ptr(hidden_q: int, hidden_scale: int, gate_q: int, gate_scale: int, T: int, H: int,
+                              E: int, k: int, scores: int, ids: int, stream: int = 0) -> int:
+    """Raw C-ABI call of the FP8 entry point with integer device pointers; returns the tk_status."""
+    return int(library().tk_gating_fused_topk_fp8(hidden_q, hidden_scale, gate_q, gate_scale, T, H, E, k, scores,
+                                                  ids, stream))
+
+
+def fused_topk_gating_fp8(hidden_q, hidden_scale, gate_q, gate_scale, top_k: int, scores=None, ids=None,
+                          stream=None):
+    """Fused gating on FP8 E4M3 inputs: ``hidden_q`` [T, H] and ``gate_q`` [E, H]
+    (expert-major) as torch.float8_e4m3fn or torch.uint8 CUDA tensors, with fp32
+    ``hidden_scale`` [T] and ``gate_scale`` [E].  Returns ``(scores, ids)``."""
+    import torch
+    fp8_types = (torch.float8_e4m3fn, torch.uint8)
+    if hidden_q.dtype not in fp8_types or gate_q.dtype not in fp8_types:
+        raise TypeError("hidden_q and gate_q must be torch.float8_e4m3fn (or their uint8 bits)")
+    if hidden_scale.dtype != torch.float32 or gate_scale.dtype != torch.float32:
+        raise TypeError("hidden_scale and gate_scale must be torch.float32")
+    if hidden_q.dim() != 2 or gate_q.dim() != 2 or hidden_q.shape[1] != gate_q.shape[1]:
+        raise ValueError(f"hidden_q {tuple(hidden_q.shape)} and gate_q {tuple(gate_q.shape)} must be [T,H] and [E,H]")
+    T, H = hidden_q.shape
+    E = gate_q.shape[0]
+    if hidden_scale.shape != (T,) or gate_scale.shape != (E,):
+        raise ValueError("hidden_scale must be [T] and gate_scale [E]")
+    tensors = (hidden_q, hidden_scale, gate_q, gate_scale)
+    if any(not t.is_cuda or t.device != hidden_q.device or not t.is_contiguous() for t in tensors):
+        raise ValueError("inputs must be contiguous CUDA tensors on one device")
+    if scores is None:
+        scores = torch.empty((T, top_k), dtype=torch.float32, device=hidden_q.device)
+    if ids is None:
+        ids = torch.empty((T, top_k), dtype=torch.int32, device=hidden_q.device)
+    with torch.cuda.device(hidden_q.device):
+        st = library().tk_gating_fused_topk_fp8(
+            hidden_q.data_ptr(), hidden_scale.data_ptr(), gate_q.data_ptr(), gate_scale.data_ptr(), T, H, E,
+            int(top_k), scores.data_ptr(), ids.data_ptr(), _stream_handle(stream, hidden_q.device))
+    _check(st, "tk_gating_fused_topk_fp8")
     return scores, ids
 
 

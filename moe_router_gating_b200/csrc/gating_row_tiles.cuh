@@ -16,6 +16,12 @@
 //   accumulating experts [256c, 256c + N_c) in tensor-memory columns from 256c;
 //   in a pair each CTA holds half of every chunk's gate columns.  The
 //   accumulator then fills tensor memory, so it is single-buffered.
+//   FP8 (E4M3) inputs (FP8 = true): the same kernel with tcgen05.mma
+//   kind::f8f6f4 (K = 32 per instruction); a 128-byte swizzle row holds 128
+//   K values instead of 64, so a K slice covers 128 elements of H with the
+//   same shared-memory footprint.  The gate is expert-major [E, H] (K-major,
+//   like the hidden rows); the epilogue multiplies each logit by its token's
+//   and its expert's scale before the selection.
 //   Balanced tail: when the last round of 256-token tiles would leave pairs
 //   idle, the remaining rows run as 128-token "half" tiles (M = 128 pair MMAs,
 //   64 rows per CTA): half the MMA cycles and three quarters of the bytes of a
@@ -78,7 +84,40 @@ struct RowTileParams {
   float* scores;
   int32_t* ids;
   uint32_t* err_word;
+  const float* hscale;  // FP8 only: per-token scales [T]
+  const float* gscale;  // FP8 only: per-expert scales [E]
 };
+
+// K elements of H per K slice: one 128-byte swizzle row of bf16 or of FP8 values.
+template <bool FP8>
+constexpr int slice_k() {
+  return FP8 ? 128 : 64;
+}
+
+// Gate descriptor of K step kk (0..3) of a slice: bf16 gate MN-major (see
+// b_desc_k_slice); FP8 gate K-major like the hidden rows (rows of 128 B, 8-row
+// groups 1024 B apart, the 32-element K step 32 B into each row).
+template <bool FP8>
+__device__ __forceinline__ uint64_t gate_desc_k_slice(uint32_t b_addr, int kk);
+
+template <bool FP8>
+__host__ __device__ constexpr uint32_t mma_idesc(uint32_t m, uint32_t n) {
+  return FP8 ? idesc_e4m3_f32(m, n) : idesc_bf16_f32(m, n, false, true);
+}
+
+// FP8: logit = accumulator * expert scale * token scale, for the 32 columns of
+// a chunk (experts e0 .. e0+31); columns past E keep a finite product of the
+// last scale and are skipped by the offer.
+template <bool FP8>
+__device__ __forceinline__ void scale_chunk(uint32_t (&r)[32], const float* gscale, int e0, int E, float hs) {
+  if constexpr (FP8) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = min(e0 + j, E - 1);
+      r[j] = __float_as_uint(__uint_as_float(r[j]) * __ldg(gscale + e) * hs);
+    }
+  }
+}
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -94,6 +133,14 @@ __device__ __forceinline__ uint64_t a_desc_k_slice(uint32_t a_stage_addr, int kk
 }
 __device__ __forceinline__ uint64_t b_desc_k_slice(uint32_t b_stage_addr, int kk) {
   return smem_desc_sw128(b_stage_addr + kk * (UMMA_K / 8) * 1024, B_BOX_BYTES, 1024);
+}
+
+template <bool FP8>
+__device__ __forceinline__ uint64_t gate_desc_k_slice(uint32_t b_addr, int kk) {
+  if constexpr (FP8)
+    return smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+  else
+    return b_desc_k_slice(b_addr, kk);
 }
 
 // Width of MMA chunk c (all but the last are N_CHUNK wide).
@@ -146,7 +193,7 @@ __device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (
   }
 }
 
-template <int KMAX, int CG>
+template <int KMAX, int CG, bool FP8>
 __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     gating_row_tiles_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_x64,
                             const __grid_constant__ CUtensorMap map_w, const RowTileParams p) {
@@ -236,18 +283,23 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
 #pragma unroll
           for (int sub = 0; sub < KB_PER_STAGE; ++sub) {
             const int slot = stage * KB_PER_STAGE + sub;
-            const int k0 = (kb + sub) * BLOCK_K;
+            const int k0 = (kb + sub) * slice_k<FP8>();
+            // gate box coordinates: bf16 [H, E] map (x = expert, y = K), FP8 [E, H] map (x = K, y = expert)
             if constexpr (kPair) {
               const uint32_t bar = map_shared_rank(smem_u32(&full[stage]), 0);
               tma_load_2d_pair(sA + slot * A_STAGE_BYTES, map_a, bar, k0, row0, pol_x);
-              for (int j = 0; j < p.b_boxes; ++j)
-                tma_load_2d_pair(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, bar,
-                                 j * B_BOX_N + (j < bpc0 ? col_a : col_b), k0, pol_w);
+              for (int j = 0; j < p.b_boxes; ++j) {
+                const int col = j * B_BOX_N + (j < bpc0 ? col_a : col_b);
+                tma_load_2d_pair(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, bar, FP8 ? k0 : col,
+                                 FP8 ? col : k0, pol_w);
+              }
             } else {
               tma_load_2d(sA + slot * A_STAGE_BYTES, &map_x, &full[stage], k0, row0, pol_x);
-              for (int j = 0; j < p.b_boxes; ++j)
-                tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage],
-                            j * B_BOX_N + (j < bpc0 ? col_a : col_b), k0, pol_w);
+              for (int j = 0; j < p.b_boxes; ++j) {
+                const int col = j * B_BOX_N + (j < bpc0 ? col_a : col_b);
+                tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], FP8 ? k0 : col,
+                            FP8 ? col : k0, pol_w);
+              }
             }
           }
           ++issued;
@@ -282,8 +334,8 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
 #pragma unroll
       for (int c = 0, box = 0; c < 2; ++c) {
         const int nc = c < p.n_chunks ? chunk_n(p, c) : N_CHUNK;
-        idesc_full[c] = idesc_bf16_f32(BLOCK_M * CG, nc, false, true);
-        idesc_half[c] = idesc_bf16_f32(BLOCK_M, nc, false, true);  // pairs: 64 rows per CTA
+        idesc_full[c] = mma_idesc<FP8>(BLOCK_M * CG, nc);
+        idesc_half[c] = mma_idesc<FP8>(BLOCK_M, nc);  // pairs: 64 rows per CTA
         b_off[c] = static_cast<uint32_t>(box * B_BOX_BYTES);
         if (c < p.n_chunks) box += chunk_boxes<CG>(p, c);
       }
@@ -318,22 +370,16 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
               for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
                 const uint32_t accumulate = ((kb + sub) | kk) != 0;
                 const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
-                if constexpr (kPair) {
-                  umma_bf16_pair(d_tmem, a_desc, b_desc_k_slice(b_addr, kk), id0, accumulate);
-                  umma_bf16_pair(d_tmem + N_CHUNK, a_desc, b_desc_k_slice(b_addr + b_off[1], kk), id1, accumulate);
-                } else {
-                  umma_bf16(d_tmem, a_desc, b_desc_k_slice(b_addr, kk), id0, accumulate);
-                  umma_bf16(d_tmem + N_CHUNK, a_desc, b_desc_k_slice(b_addr + b_off[1], kk), id1, accumulate);
-                }
+                umma<FP8, kPair>(d_tmem, a_desc, gate_desc_k_slice<FP8>(b_addr, kk), id0, accumulate);
+                umma<FP8, kPair>(d_tmem + N_CHUNK, a_desc, gate_desc_k_slice<FP8>(b_addr + b_off[1], kk), id1,
+                                 accumulate);
               }
             } else {
 #pragma unroll
               for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
                 const uint32_t accumulate = ((kb + sub) | kk) != 0;
-                if constexpr (kPair)
-                  umma_bf16_pair(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), id0, accumulate);
-                else
-                  umma_bf16(d_tmem, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), id0, accumulate);
+                umma<FP8, kPair>(d_tmem, a_desc_k_slice(a_addr, kk), gate_desc_k_slice<FP8>(b_addr, kk), id0,
+                                 accumulate);
               }
             }
           }
@@ -382,6 +428,12 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       RowTopK<KMAX> top;
       top.reset();
       const uint32_t acc_addr = lane_base + buf * p.acc_stride;
+      float hs = 1.0f;  // FP8: this row's token scale
+      if constexpr (FP8) {
+        const int64_t my_row = w.half ? static_cast<int64_t>(w.row0) + rank * (BLOCK_M / 2) + (quad & 1) * 32 + lane
+                                      : static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
+        hs = my_row < p.T ? __ldg(p.hscale + my_row) : 0.0f;
+      }
       // full tiles: one pass over columns [0, E); half tiles: one per chunk
       const int passes = w.half ? p.n_chunks : 1;
       for (int c = 0; c < passes; ++c) {
@@ -399,8 +451,12 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           tmem_ld_32(chunk_addr + c0, r0);
           if (second) tmem_ld_32(chunk_addr + c0 + 32, r1);
           tmem_ld_wait();
+          scale_chunk<FP8>(r0, p.gscale, col_base + c0, p.E, hs);
           offer_chunk(top, r0, c0, ncols, col_base);
-          if (second) offer_chunk(top, r1, c0 + 32, ncols, col_base);
+          if (second) {
+            scale_chunk<FP8>(r1, p.gscale, col_base + c0 + 32, p.E, hs);
+            offer_chunk(top, r1, c0 + 32, ncols, col_base);
+          }
         }
       }
       // the accumulator buffer may be overwritten once every epilogue warp of

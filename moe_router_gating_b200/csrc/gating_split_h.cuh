@@ -25,6 +25,10 @@
 // once per 256-expert column range: each pass pushes and reduces its columns
 // and the owners keep their running top-k lists across passes.
 //
+// FP8 = true: E4M3 inputs as in the row-tile kernel (kind::f8f6f4, K-major
+// expert-major gate, 128 K values per slice); owners scale the summed logits
+// by the token's and the expert's scale before selecting.
+//
 // Nothing but scores and ids is written to global memory.
 #pragma once
 
@@ -61,9 +65,11 @@ struct SplitHParams {
   float* scores;
   int32_t* ids;
   uint32_t* err_word;
+  const float* hscale;  // FP8 only: per-token scales [T]
+  const float* gscale;  // FP8 only: per-expert scales [E]
 };
 
-template <int KMAX, int C>
+template <int KMAX, int C, bool FP8>
 __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     gating_split_h_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                           const SplitHParams p) {
@@ -125,10 +131,12 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
         mbar_arrive_expect_tx(&full[stage], n_sub * slice_tx);
         for (int sub = 0; sub < n_sub; ++sub) {
           const int slot = stage * p.kps + sub;
-          const int k0 = (kb + sub) * BLOCK_K;
+          const int k0 = (kb + sub) * slice_k<FP8>();
           tma_load_2d(sA + slot * A_STAGE_BYTES, &map_x, &full[stage], k0, tile * BLOCK_M, pol_x);
+          // gate box coordinates: bf16 [H, E] map (x = expert, y = K), FP8 [E, H] map (x = K, y = expert)
           for (int j = 0; j < p.b_boxes; ++j)
-            tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], j * B_BOX_N, k0, pol_w);
+            tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], FP8 ? k0 : j * B_BOX_N,
+                        FP8 ? j * B_BOX_N : k0, pol_w);
         }
         ++issued;
         if (++stage == static_cast<uint32_t>(p.stages)) {
@@ -151,8 +159,8 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       // chunk c: N = min(256, n_pad - 256c); its gate boxes start at box 4c
-      const uint32_t idesc0 = idesc_bf16_f32(BLOCK_M, min(p.n_pad, 256), false, true);
-      const uint32_t idesc1 = idesc_bf16_f32(BLOCK_M, p.n_pad > 256 ? p.n_pad - 256 : 256, false, true);
+      const uint32_t idesc0 = mma_idesc<FP8>(BLOCK_M, min(p.n_pad, 256));
+      const uint32_t idesc1 = mma_idesc<FP8>(BLOCK_M, p.n_pad > 256 ? p.n_pad - 256 : 256);
       const bool two_chunks = p.n_chunks > 1;
       uint32_t stage = 0, phase = 0;
       bool ok = true;
@@ -172,15 +180,16 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
             for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
               const uint32_t accumulate = (kb + sub != kb0) | kk;
               const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
-              umma_bf16(tmem_base, a_desc, b_desc_k_slice(b_addr, kk), idesc0, accumulate);
-              umma_bf16(tmem_base + N_CHUNK, a_desc, b_desc_k_slice(b_addr + (N_CHUNK / B_BOX_N) * B_BOX_BYTES, kk),
-                        idesc1, accumulate);
+              umma<FP8, false>(tmem_base, a_desc, gate_desc_k_slice<FP8>(b_addr, kk), idesc0, accumulate);
+              umma<FP8, false>(tmem_base + N_CHUNK, a_desc,
+                               gate_desc_k_slice<FP8>(b_addr + (N_CHUNK / B_BOX_N) * B_BOX_BYTES, kk), idesc1,
+                               accumulate);
             }
           } else {
 #pragma unroll
             for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
-              umma_bf16(tmem_base, a_desc_k_slice(a_addr, kk), b_desc_k_slice(b_addr, kk), idesc0,
-                        (kb + sub != kb0) | kk);
+              umma<FP8, false>(tmem_base, a_desc_k_slice(a_addr, kk), gate_desc_k_slice<FP8>(b_addr, kk), idesc0,
+                               (kb + sub != kb0) | kk);
           }
         }
         umma_commit(&empty[stage]);
@@ -281,6 +290,8 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
 
     // ---------------- reduce owned rows of this pass into the running top-k ----------------
     if (active) {
+      float hs = 1.0f;  // FP8: the row's token scale
+      if constexpr (FP8) hs = __ldg(p.hscale + static_cast<int64_t>(tile) * BLOCK_M + static_cast<int>(r) + C * slot);
       // segment `seg` takes every group-th float4 of the row: consecutive lanes
       // read consecutive 16-byte words (no bank conflicts), and each thread still
       // offers its columns in increasing order
@@ -296,6 +307,13 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
           acc.y += v[q].y;
           acc.z += v[q].z;
           acc.w += v[q].w;
+        }
+        if constexpr (FP8) {  // expert scales of columns past E are never offered
+          const int e = col0 + c;
+          acc.x = acc.x * __ldg(p.gscale + min(e, p.E - 1)) * hs;
+          acc.y = acc.y * __ldg(p.gscale + min(e + 1, p.E - 1)) * hs;
+          acc.z = acc.z * __ldg(p.gscale + min(e + 2, p.E - 1)) * hs;
+          acc.w = acc.w * __ldg(p.gscale + min(e + 3, p.E - 1)) * hs;
         }
         top.offer(acc.x, col0 + c);
         if (c + 1 < pass_cols) top.offer(acc.y, col0 + c + 1);

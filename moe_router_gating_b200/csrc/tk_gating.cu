@@ -195,6 +195,21 @@ bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D uint8 (FP8 E4M3 bits) row-major [rows, cols] map with a (box_cols x
+// box_rows) box, 128-byte swizzle: a box row of 128 values is one swizzle row.
+bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estrides[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estrides,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Per-device facts and one-time kernel set-up, filled on the first call made with
 // that device current: compute capability, SM count, the device address of the
 // error word, every kernel's shared-memory limit (set to the maximum once, so no
@@ -218,14 +233,21 @@ bool set_smem_limit(Kernel kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem) == cudaSuccess;
 }
 
+template <int KMAX, bool FP8>
+bool set_up_kernels_of() {
+  bool ok = set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 1, FP8>) &&
+            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2, FP8>) &&
+            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 2, FP8>) &&
+            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 4, FP8>) &&
+            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 8, FP8>) &&
+            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 16, FP8>);
+  return ok && cudaFuncSetAttribute(tkg::gating_split_h_kernel<KMAX, 16, FP8>,
+                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+}
+
 template <int KMAX>
 bool set_up_kernels() {
-  bool ok = set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 1>) &&
-            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2>) &&
-            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 2>) && set_smem_limit(tkg::gating_split_h_kernel<KMAX, 4>) &&
-            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 8>) && set_smem_limit(tkg::gating_split_h_kernel<KMAX, 16>);
-  return ok && cudaFuncSetAttribute(tkg::gating_split_h_kernel<KMAX, 16>,
-                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  return set_up_kernels_of<KMAX, false>() && set_up_kernels_of<KMAX, true>();
 }
 
 // Clusters of each size 2^i (i = 1..4) of full-shared-memory CTAs that the
@@ -247,8 +269,8 @@ ClusterCapacity measure_cluster_capacity(int num_sms) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    cudaError_t e = C == 16 ? cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 16>, &cfg)
-                            : cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 8>, &cfg);
+    cudaError_t e = C == 16 ? cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 16, false>, &cfg)
+                            : cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 8, false>, &cfg);
     if (e != cudaSuccess) {
       cudaGetLastError();
       n = 0;
@@ -295,10 +317,10 @@ const DeviceState* device_state() {
   return &d;
 }
 
-template <int KMAX, int CG>
+template <int KMAX, int CG, bool FP8>
 tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
                            const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
-  auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG>;
+  auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG, FP8>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
@@ -315,10 +337,10 @@ tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, cons
   return TK_OK;
 }
 
-template <int KMAX, int C>
+template <int KMAX, int C, bool FP8>
 tk_status launch_split_h_c(const tk_gating_plan& plan, const CUtensorMap& mx, const CUtensorMap& mw,
                            const tkg::SplitHParams& prm, cudaStream_t stream) {
-  auto kernel = tkg::gating_split_h_kernel<KMAX, C>;
+  auto kernel = tkg::gating_split_h_kernel<KMAX, C, FP8>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
@@ -335,25 +357,93 @@ tk_status launch_split_h_c(const tk_gating_plan& plan, const CUtensorMap& mx, co
   return TK_OK;
 }
 
-template <int KMAX>
+template <int KMAX, bool FP8>
 tk_status launch_split_h(const tk_gating_plan& plan, int max_cluster, const CUtensorMap& mx, const CUtensorMap& mw,
                          const tkg::SplitHParams& prm, cudaStream_t stream) {
   int C = plan.cluster;
   while (C > max_cluster) C >>= 1;  // the largest cluster the device co-schedules
   switch (C) {
-    case 16: return launch_split_h_c<KMAX, 16>(plan, mx, mw, prm, stream);
-    case 8: return launch_split_h_c<KMAX, 8>(plan, mx, mw, prm, stream);
-    case 4: return launch_split_h_c<KMAX, 4>(plan, mx, mw, prm, stream);
-    case 2: return launch_split_h_c<KMAX, 2>(plan, mx, mw, prm, stream);
+    case 16: return launch_split_h_c<KMAX, 16, FP8>(plan, mx, mw, prm, stream);
+    case 8: return launch_split_h_c<KMAX, 8, FP8>(plan, mx, mw, prm, stream);
+    case 4: return launch_split_h_c<KMAX, 4, FP8>(plan, mx, mw, prm, stream);
+    case 2: return launch_split_h_c<KMAX, 2, FP8>(plan, mx, mw, prm, stream);
     default: return TK_ERR_UNSUPPORTED;
   }
 }
 
-template <int KMAX>
+template <int KMAX, bool FP8>
 tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
                              const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
-  if (pl.variant == TK_VARIANT_ROW_PAIRS) return launch_row_tiles<KMAX, 2>(pl, mx, mx64, mw, prm, stream);
-  return launch_row_tiles<KMAX, 1>(pl, mx, mx64, mw, prm, stream);
+  if (pl.variant == TK_VARIANT_ROW_PAIRS) return launch_row_tiles<KMAX, 2, FP8>(pl, mx, mx64, mw, prm, stream);
+  return launch_row_tiles<KMAX, 1, FP8>(pl, mx, mx64, mw, prm, stream);
+}
+
+// Launch the planned kernel on encoded maps.  FP8: hscale / gscale are the
+// per-token and per-expert scales (unused for bf16).
+template <bool FP8>
+tk_status launch_planned(const tk_gating_plan& pl, const DeviceState* dev, const CUtensorMap& mx,
+                         const CUtensorMap& mx64, const CUtensorMap& mw, int64_t T, int64_t H, int64_t E, int32_t k,
+                         float* scores, int32_t* ids, const float* hscale, const float* gscale, cudaStream_t stream) {
+  uint32_t* err = dev->err_word;
+  if (pl.variant == TK_VARIANT_SPLIT_H) {
+    tkg::SplitHParams sp;
+    sp.T = static_cast<int32_t>(T);
+    sp.H = static_cast<int32_t>(H);
+    sp.E = static_cast<int32_t>(E);
+    sp.k = k;
+    sp.n_pad = pl.n_pad;
+    sp.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
+    sp.kps = pl.slices_per_stage;
+    sp.num_tiles = pl.num_tiles;
+    sp.k_blocks = pl.k_blocks;
+    sp.stages = pl.stages;
+    sp.b_boxes = (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+    sp.row_stride = split_row_stride(E);
+    sp.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
+    sp.timeout_ns = g_timeout_ns;
+    sp.scores = scores;
+    sp.ids = ids;
+    sp.err_word = err;
+    sp.hscale = hscale;
+    sp.gscale = gscale;
+    const int mc = dev->max_split_cluster;
+    if (k <= 1) return launch_split_h<1, FP8>(pl, mc, mx, mw, sp, stream);
+    if (k <= 2) return launch_split_h<2, FP8>(pl, mc, mx, mw, sp, stream);
+    if (k <= 4) return launch_split_h<4, FP8>(pl, mc, mx, mw, sp, stream);
+    if (k <= 8) return launch_split_h<8, FP8>(pl, mc, mx, mw, sp, stream);
+    if (k <= 16) return launch_split_h<16, FP8>(pl, mc, mx, mw, sp, stream);
+    return launch_split_h<32, FP8>(pl, mc, mx, mw, sp, stream);
+  }
+
+  tkg::RowTileParams prm;
+  prm.T = static_cast<int32_t>(T);
+  prm.H = static_cast<int32_t>(H);
+  prm.E = static_cast<int32_t>(E);
+  prm.k = k;
+  prm.n_pad = pl.n_pad;
+  prm.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
+  prm.acc_stride = round_up(pl.n_pad, 32);
+  prm.acc_bufs = 2 * prm.acc_stride <= 512 ? 2 : 1;
+  prm.num_tiles = pl.num_tiles;
+  prm.num_half = pl.num_half_tiles;
+  prm.k_blocks = pl.k_blocks;
+  prm.stages = pl.stages;
+  prm.b_boxes = pl.variant == TK_VARIANT_ROW_PAIRS ? pl.n_pad / 2 / tkg::B_BOX_N
+                                                   : (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+  prm.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
+  prm.timeout_ns = g_timeout_ns;
+  prm.scores = scores;
+  prm.ids = ids;
+  prm.err_word = err;
+  prm.hscale = hscale;
+  prm.gscale = gscale;
+
+  if (k <= 1) return launch_row_variant<1, FP8>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 2) return launch_row_variant<2, FP8>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 4) return launch_row_variant<4, FP8>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 8) return launch_row_variant<8, FP8>(pl, mx, mx64, mw, prm, stream);
+  if (k <= 16) return launch_row_variant<16, FP8>(pl, mx, mx64, mw, prm, stream);
+  return launch_row_variant<32, FP8>(pl, mx, mx64, mw, prm, stream);
 }
 
 tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int64_t H, int64_t E, int32_t k,
@@ -378,62 +468,43 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
                                                 tkg::BLOCK_K, tkg::BLOCK_M / 2)) ||
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
-  uint32_t* err = dev->err_word;
+  return launch_planned<false>(pl, dev, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, stream);
+}
 
-  if (pl.variant == TK_VARIANT_SPLIT_H) {
-    tkg::SplitHParams sp;
-    sp.T = static_cast<int32_t>(T);
-    sp.H = static_cast<int32_t>(H);
-    sp.E = static_cast<int32_t>(E);
-    sp.k = k;
-    sp.n_pad = pl.n_pad;
-    sp.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
-    sp.kps = pl.slices_per_stage;
-    sp.num_tiles = pl.num_tiles;
-    sp.k_blocks = pl.k_blocks;
-    sp.stages = pl.stages;
-    sp.b_boxes = (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
-    sp.row_stride = split_row_stride(E);
-    sp.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
-    sp.timeout_ns = g_timeout_ns;
-    sp.scores = scores;
-    sp.ids = ids;
-    sp.err_word = err;
-    if (k <= 1) return launch_split_h<1>(pl, dev->max_split_cluster, mx, mw, sp, stream);
-    if (k <= 2) return launch_split_h<2>(pl, dev->max_split_cluster, mx, mw, sp, stream);
-    if (k <= 4) return launch_split_h<4>(pl, dev->max_split_cluster, mx, mw, sp, stream);
-    if (k <= 8) return launch_split_h<8>(pl, dev->max_split_cluster, mx, mw, sp, stream);
-    if (k <= 16) return launch_split_h<16>(pl, dev->max_split_cluster, mx, mw, sp, stream);
-    return launch_split_h<32>(pl, dev->max_split_cluster, mx, mw, sp, stream);
-  }
+// FP8 sizes: H a multiple of 16 (16-byte rows of 8-bit values); E and k as bf16.
+tk_status validate_sizes_fp8(int64_t T, int64_t H, int64_t E, int32_t k) {
+  if (T < 0 || H < 1 || E < 1 || k < 1 || k > E) return TK_ERR_INVALID_ARG;
+  if (H % 16 != 0) return TK_ERR_UNSUPPORTED;
+  return validate_sizes(T, H / 2, E, k);
+}
 
-  tkg::RowTileParams prm;
-  prm.T = static_cast<int32_t>(T);
-  prm.H = static_cast<int32_t>(H);
-  prm.E = static_cast<int32_t>(E);
-  prm.k = k;
-  prm.n_pad = pl.n_pad;
-  prm.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
-  prm.acc_stride = round_up(pl.n_pad, 32);
-  prm.acc_bufs = 2 * prm.acc_stride <= 512 ? 2 : 1;
-  prm.num_tiles = pl.num_tiles;
-  prm.num_half = pl.num_half_tiles;
-  prm.k_blocks = pl.k_blocks;
-  prm.stages = pl.stages;
-  prm.b_boxes = pl.variant == TK_VARIANT_ROW_PAIRS ? pl.n_pad / 2 / tkg::B_BOX_N
-                                                   : (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
-  prm.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
-  prm.timeout_ns = g_timeout_ns;
-  prm.scores = scores;
-  prm.ids = ids;
-  prm.err_word = err;
+tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale, const void* gate_q,
+                                const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k, float* scores,
+                                int32_t* ids, cudaStream_t stream) {
+  tk_status st = validate_sizes_fp8(T, H, E, k);
+  if (st != TK_OK) return st;
+  if (T == 0) return TK_OK;
+  if (!hidden_q || !hidden_scale || !gate_q || !gate_scale || !scores || !ids) return TK_ERR_INVALID_ARG;
+  if (!aligned16(hidden_q) || !aligned16(gate_q) || !aligned16(scores) || !aligned16(ids) ||
+      !aligned16(hidden_scale) || !aligned16(gate_scale))
+    return TK_ERR_ALIGNMENT;
+  const DeviceState* dev = device_state();
+  if (dev == nullptr) return TK_ERR_CUDA;
+  if (dev->status != TK_OK) return dev->status;
+  // a K slice of 128 FP8 values occupies what 64 bf16 values do: plan on H / 2
+  tk_gating_plan pl;
+  st = plan_impl(T, H / 2, E, k, dev->num_sms, dev->capacity, &pl);
+  if (st != TK_OK) return st;
 
-  if (k <= 1) return launch_row_variant<1>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 2) return launch_row_variant<2>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 4) return launch_row_variant<4>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 8) return launch_row_variant<8>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 16) return launch_row_variant<16>(pl, mx, mx64, mw, prm, stream);
-  return launch_row_variant<32>(pl, mx, mx64, mw, prm, stream);
+  CUtensorMap mx, mx64, mw;
+  std::memset(&mx64, 0, sizeof(mx64));
+  const uint32_t kslice = 2 * tkg::BLOCK_K;  // 128 values: one 128-byte swizzle row
+  if (!encode_2d_u8(&mx, hidden_q, static_cast<uint64_t>(T), static_cast<uint64_t>(H), kslice, tkg::BLOCK_M) ||
+      (pl.num_half_tiles > 0 &&
+       !encode_2d_u8(&mx64, hidden_q, static_cast<uint64_t>(T), static_cast<uint64_t>(H), kslice, tkg::BLOCK_M / 2)) ||
+      !encode_2d_u8(&mw, gate_q, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kslice, tkg::B_BOX_N))
+    return TK_ERR_CUDA;
+  return launch_planned<true>(pl, dev, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, stream);
 }
 
 }  // namespace
@@ -466,6 +537,13 @@ tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* gate_we
       cudaMemcpyAsync(ids_host, ids_dev, out_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return TK_ERR_CUDA;
   return TK_OK;
+}
+
+tk_status tk_gating_fused_topk_fp8(const void* hidden_q, const float* hidden_scale, const void* gate_q,
+                                   const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k, float* scores,
+                                   int32_t* ids, void* stream) {
+  return fused_topk_fp8_device(hidden_q, hidden_scale, gate_q, gate_scale, T, H, E, k, scores, ids,
+                               static_cast<cudaStream_t>(stream));
 }
 
 tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan) {

@@ -148,3 +148,13 @@ def test_plan_large_expert_counts():
     assert p["variant"] == 2 and p["slices_per_stage"] == 1 and p["tmem_cols"] == 512
     p = tk.make_plan(4096, 7168, 256, 8, 148)
     assert p["slices_per_stage"] == 2
+
+
+def test_fp8_entry_point_rejects_before_cuda():
+    f = tk.fused_topk_gating_fp8_ptr
+    assert f(16, 16, 16, 16, 8, 72, 16, 2, 16, 16) == tk.TK_ERR_UNSUPPORTED        # H % 16 != 0
+    assert f(16, 16, 16, 16, 8, 64, 16, 17, 16, 16) == tk.TK_ERR_INVALID_ARG       # k > E
+    assert f(16, 16, 16, 16, 8, 64, 520, 2, 16, 16) == tk.TK_ERR_UNSUPPORTED       # E > 512
+    assert f(16, 0, 16, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_INVALID_ARG         # null scale
+    assert f(16, 20, 16, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_ALIGNMENT          # scale not 16-byte aligned
+    assert f(0, 0, 0, 0, 0, 64, 16, 2, 0, 0) == tk.TK_OK                             # T == 0

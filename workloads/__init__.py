@@ -196,8 +196,10 @@ def fp8_inputs(wl: "RouterWorkload"):
     """FP8 versions of a workload's inputs: the bf16 hidden rows quantized per token,
     the bf16 gate quantized per expert and stored expert-major [E, H].
     Returns (hidden_q [T, H], hidden_scale [T], gate_q [E, H], gate_scale [E])."""
-    xq, xs = quantize_e4m3_rows(bf16_to_f64(wl.hidden()).astype(np.float32))
-    wq, ws = quantize_e4m3_rows(bf16_to_f64(wl.gate_weight()).T.astype(np.float32))
+    def to_f32(bits):  # exact bf16 -> fp32 widening
+        return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+    xq, xs = quantize_e4m3_rows(to_f32(wl.hidden()))
+    wq, ws = quantize_e4m3_rows(np.ascontiguousarray(to_f32(wl.gate_weight()).T))
     return xq, xs, wq, ws
 
 
