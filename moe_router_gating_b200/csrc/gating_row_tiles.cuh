@@ -111,10 +111,22 @@ __host__ __device__ constexpr uint32_t mma_idesc(uint32_t m, uint32_t n) {
 template <bool FP8>
 __device__ __forceinline__ void scale_chunk(uint32_t (&r)[32], const float* gscale, int e0, int E, float hs) {
   if constexpr (FP8) {
+    if (e0 + 32 <= E) {  // e0 is a multiple of 32 and gscale 16-byte aligned: eight 16-byte loads
+      const float4* g4 = reinterpret_cast<const float4*>(gscale + e0);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int e = min(e0 + j, E - 1);
-      r[j] = __float_as_uint(__uint_as_float(r[j]) * __ldg(gscale + e) * hs);
+      for (int q = 0; q < 8; ++q) {
+        const float4 g = __ldg(g4 + q);
+        r[4 * q + 0] = __float_as_uint(__uint_as_float(r[4 * q + 0]) * g.x * hs);
+        r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) * g.y * hs);
+        r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) * g.z * hs);
+        r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) * g.w * hs);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int e = min(e0 + j, E - 1);
+        r[j] = __float_as_uint(__uint_as_float(r[j]) * __ldg(gscale + e) * hs);
+      }
     }
   }
 }
