@@ -57,7 +57,7 @@ typedef enum {
 } tk_status;
 
 /* Limits of the fused kernels. */
-#define TK_GATING_MAX_EXPERTS 512
+#define TK_GATING_MAX_EXPERTS 1024
 #define TK_GATING_MAX_TOPK 32
 
 /*
@@ -68,7 +68,7 @@ typedef enum {
  *                `hidden_states @ gate_weight`; expert e is column e).
  *   T            tokens, T >= 0.  T == 0 returns TK_OK and launches nothing.
  *   H            hidden size, H >= 8 and H % 8 == 0 (16-byte row pitch).
- *   E            experts, 16 <= E <= 512 and E % 8 == 0.
+ *   E            experts, 16 <= E <= 1024 and E % 8 == 0.
  *   k            experts kept per token, 1 <= k <= min(E, 32).
  *   scores       device, out fp32 [T, k] row-major.
  *   ids          device, out int32 [T, k] row-major.
@@ -77,7 +77,7 @@ typedef enum {
  * Errors:
  *   TK_ERR_INVALID_ARG   T < 0, H < 1, E < 1, k < 1, k > E, or a null pointer
  *                        when T > 0;
- *   TK_ERR_UNSUPPORTED   H or E not a multiple of 8, E < 16, E > 512, k > 32,
+ *   TK_ERR_UNSUPPORTED   H or E not a multiple of 8, E < 16, E > 1024, k > 32,
  *                        T >= 2^31 - 128, or the current device is not sm_100;
  *   TK_ERR_ALIGNMENT     a pointer is not 16-byte aligned;
  *   TK_ERR_CUDA          a CUDA call (device query, descriptor encode, launch)
@@ -166,6 +166,7 @@ typedef struct {
   int32_t tmem_cols;    /* tensor-memory columns allocated per CTA */
   int32_t num_half_tiles; /* CTA pairs: 128-token tiles after the full ones (balanced last round) */
   int32_t slices_per_stage; /* 64-wide K slices per ring stage */
+  int32_t expert_groups;  /* groups of at most 512 experts, computed one after the other per tile (1 or 2) */
 } tk_gating_plan;
 
 /*

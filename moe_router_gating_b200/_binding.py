@@ -31,7 +31,7 @@ class TkGatingError(RuntimeError):
 class _Plan(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in (
         "variant", "block_m", "n_pad", "num_tiles", "k_blocks", "split_h", "stages", "grid", "cluster",
-        "threads", "smem_bytes", "tmem_cols", "num_half_tiles", "slices_per_stage")]
+        "threads", "smem_bytes", "tmem_cols", "num_half_tiles", "slices_per_stage", "expert_groups")]
 
 
 class _RoutePlan(ctypes.Structure):

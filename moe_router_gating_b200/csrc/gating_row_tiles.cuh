@@ -16,6 +16,11 @@
 //   accumulating experts [256c, 256c + N_c) in tensor-memory columns from 256c;
 //   in a pair each CTA holds half of every chunk's gate columns.  The
 //   accumulator then fills tensor memory, so it is single-buffered.
+//   More than 512 experts (up to 1024): the experts form two groups of at most
+//   512, and every tile is two work items, one per group, back to back on the
+//   same CTA (pair); the epilogue keeps its rows' top-k lists across the two
+//   items and stores after the second.  The hidden tile is streamed once per
+//   group.
 //   FP8 (E4M3) inputs (FP8 = true): the same kernel with tcgen05.mma
 //   kind::f8f6f4 (K = 32 per instruction); a 128-byte swizzle row holds 128
 //   K values instead of 64, so a K slice covers 128 elements of H with the
@@ -70,15 +75,15 @@ constexpr int N_CHUNK = 256;                            // MMA N per instruction
 
 struct RowTileParams {
   int32_t T, H, E, k;
-  int32_t n_pad;        // total MMA N (CG=1: E rounded up to 16; CG=2: a multiple of 128, <= 512)
-  int32_t n_chunks;     // ceil(n_pad / 256): MMAs per K step
+  int32_t n_pad;        // total MMA N over all experts (CG=1: E rounded up to 16; CG=2: a multiple of 128)
+  int32_t e_groups;     // expert groups of at most 512 (1 or 2; the kernel's EG); group g from expert 512 g
   int32_t acc_stride;   // TMEM columns between accumulator buffers
   int32_t acc_bufs;     // accumulator buffers in TMEM (2, or 1 when n_pad > 256)
   int32_t num_tiles;    // full tiles of BLOCK_M * CG rows, starting at row 0
   int32_t num_half;     // pairs only: half tiles of BLOCK_M rows after the full tiles
   int32_t k_blocks;
   int32_t stages;       // ring stages of KB_PER_STAGE K slices
-  int32_t b_boxes;      // gate boxes per K slice loaded by each CTA
+  int32_t b_boxes;      // gate boxes per K slice and CTA in the ring (group 0's count, the largest)
   uint32_t tmem_cols;
   uint64_t timeout_ns;
   float* scores;
@@ -155,15 +160,32 @@ __device__ __forceinline__ uint64_t gate_desc_k_slice(uint32_t b_addr, int kk) {
     return b_desc_k_slice(b_addr, kk);
 }
 
-// Width of MMA chunk c (all but the last are N_CHUNK wide).
-__device__ __forceinline__ int chunk_n(const RowTileParams& p, int c) {
-  return c + 1 < p.n_chunks ? N_CHUNK : p.n_pad - N_CHUNK * (p.n_chunks - 1);
+constexpr int E_GROUP = 512;  // experts per group: the MMA N that fits tensor memory
+
+// The MMA shape of expert group g: n_pad columns in n_chunks chunks.
+struct GroupShape {
+  int e0;        // first expert of the group
+  int n_pad;     // MMA N of the group
+  int n_chunks;  // ceil(n_pad / 256)
+};
+
+__device__ __forceinline__ GroupShape group_shape(const RowTileParams& p, int g) {
+  GroupShape s;
+  s.e0 = g * E_GROUP;
+  s.n_pad = g == 0 ? min(p.n_pad, E_GROUP) : p.n_pad - E_GROUP;
+  s.n_chunks = (s.n_pad + N_CHUNK - 1) / N_CHUNK;
+  return s;
+}
+
+// Width of MMA chunk c of a group (all but the last are N_CHUNK wide).
+__device__ __forceinline__ int chunk_n(const GroupShape& s, int c) {
+  return c + 1 < s.n_chunks ? N_CHUNK : s.n_pad - N_CHUNK * (s.n_chunks - 1);
 }
 
 // Gate boxes (64 experts each) of chunk c that one CTA stages per K slice.
 template <int CG>
-__device__ __forceinline__ int chunk_boxes(const RowTileParams& p, int c) {
-  return (chunk_n(p, c) / CG + B_BOX_N - 1) / B_BOX_N;
+__device__ __forceinline__ int chunk_boxes(const GroupShape& s, int c) {
+  return (chunk_n(s, c) / CG + B_BOX_N - 1) / B_BOX_N;
 }
 
 // The i-th tile of a CTA (or pair) `unit` out of `units`: full tiles round-robin,
@@ -171,10 +193,14 @@ __device__ __forceinline__ int chunk_boxes(const RowTileParams& p, int c) {
 struct TileWork {
   int row0;   // first token row of the tile (pair tile: of the pair)
   bool half;  // 128-token pair tile
+  int eg;     // expert group of this work item
 };
 
-template <int CG>
-__device__ __forceinline__ bool tile_work(const RowTileParams& p, int unit, int units, int i, TileWork& w) {
+template <int CG, int EG>
+__device__ __forceinline__ bool tile_work(const RowTileParams& p, int unit, int units, int item, TileWork& w) {
+  // every tile is EG (1 or 2) consecutive work items, one per expert group
+  const int i = EG == 1 ? item : item >> 1;
+  w.eg = EG == 1 ? 0 : item & 1;
   const int n_full = unit < p.num_tiles ? (p.num_tiles - 1 - unit) / units + 1 : 0;
   if (i < n_full) {
     w.row0 = (unit + i * units) * (BLOCK_M * CG);
@@ -205,7 +231,10 @@ __device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (
   }
 }
 
-template <int KMAX, int CG, bool FP8>
+// EG: expert groups (compile time, so that the single-group kernel carries no
+// group bookkeeping: kept at run time it cost ~4% of the 65536-token kernel's
+// cycles).
+template <int KMAX, int CG, bool FP8, int EG>
 __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     gating_row_tiles_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_x64,
                             const __grid_constant__ CUtensorMap map_w, const RowTileParams p) {
@@ -273,17 +302,23 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       const uint64_t pol_w = l2_policy_evict_last();   // gate: re-read by every tile
       // gate box j of a K slice starts at column j * 64 + (j < bpc0 ? col_a : col_b): this
       // CTA's share of chunk 0 (bpc0 boxes), then of chunk 1 (starting at expert 256)
-      const int bpc0 = chunk_boxes<CG>(p, 0);
-      const int col_a = static_cast<int>(rank) * (chunk_n(p, 0) / CG);
-      const int col_b = p.n_chunks > 1 ? N_CHUNK + static_cast<int>(rank) * (chunk_n(p, 1) / CG) - bpc0 * B_BOX_N : 0;
       uint32_t stage = 0, phase = 0;
       int issued = 0;
       bool ok = true;
       TileWork w;
-      for (int item = 0; ok && tile_work<CG>(p, unit, units, item, w); ++item) {
+      for (int item = 0; ok && tile_work<CG, EG>(p, unit, units, item, w); ++item) {
         const int cta_rows = w.half ? BLOCK_M / 2 : BLOCK_M;  // hidden rows this CTA stages
         const int row0 = w.row0 + static_cast<int>(rank) * cta_rows;
-        const uint32_t stage_tx = KB_PER_STAGE * CG * (cta_rows * BLOCK_K * 2 + p.b_boxes * B_BOX_BYTES);
+        // this work item's gate boxes: box j of a K slice starts at expert
+        // j * 64 + (j < bpc0 ? col_a : col_b), this CTA's share of chunk 0 (bpc0
+        // boxes), then of chunk 1 (from the group's expert 256)
+        const GroupShape gs = group_shape(p, w.eg);
+        const int bpc0 = chunk_boxes<CG>(gs, 0);
+        const int boxes = bpc0 + (gs.n_chunks > 1 ? chunk_boxes<CG>(gs, 1) : 0);
+        const int col_a = gs.e0 + static_cast<int>(rank) * (chunk_n(gs, 0) / CG);
+        const int col_b =
+            gs.n_chunks > 1 ? gs.e0 + N_CHUNK + static_cast<int>(rank) * (chunk_n(gs, 1) / CG) - bpc0 * B_BOX_N : 0;
+        const uint32_t stage_tx = KB_PER_STAGE * CG * (cta_rows * BLOCK_K * 2 + boxes * B_BOX_BYTES);
         const CUtensorMap* map_a = w.half ? &map_x64 : &map_x;
         // K slices past H (when k_blocks is odd) are out of bounds: TMA fills zeros
         for (int kb = 0; kb < p.k_blocks; kb += KB_PER_STAGE) {
@@ -300,14 +335,14 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
             if constexpr (kPair) {
               const uint32_t bar = map_shared_rank(smem_u32(&full[stage]), 0);
               tma_load_2d_pair(sA + slot * A_STAGE_BYTES, map_a, bar, k0, row0, pol_x);
-              for (int j = 0; j < p.b_boxes; ++j) {
+              for (int j = 0; j < boxes; ++j) {
                 const int col = j * B_BOX_N + (j < bpc0 ? col_a : col_b);
                 tma_load_2d_pair(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, bar, FP8 ? k0 : col,
                                  FP8 ? col : k0, pol_w);
               }
             } else {
               tma_load_2d(sA + slot * A_STAGE_BYTES, &map_x, &full[stage], k0, row0, pol_x);
-              for (int j = 0; j < p.b_boxes; ++j) {
+              for (int j = 0; j < boxes; ++j) {
                 const int col = j * B_BOX_N + (j < bpc0 ? col_a : col_b);
                 tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], FP8 ? k0 : col,
                             FP8 ? col : k0, pol_w);
@@ -340,27 +375,21 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ---------------- MMA issuer ----------------
-      // per chunk: instruction descriptor (full and half tiles) and the offset of
-      // its gate boxes within a K slice
-      uint32_t idesc_full[2], idesc_half[2], b_off[2];
-#pragma unroll
-      for (int c = 0, box = 0; c < 2; ++c) {
-        const int nc = c < p.n_chunks ? chunk_n(p, c) : N_CHUNK;
-        idesc_full[c] = mma_idesc<FP8>(BLOCK_M * CG, nc);
-        idesc_half[c] = mma_idesc<FP8>(BLOCK_M, nc);  // pairs: 64 rows per CTA
-        b_off[c] = static_cast<uint32_t>(box * B_BOX_BYTES);
-        if (c < p.n_chunks) box += chunk_boxes<CG>(p, c);
-      }
-      const bool two_chunks = p.n_chunks > 1;
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
       TileWork w;
-      for (; ok && tile_work<CG>(p, unit, units, local, w); ++local) {
+      for (; ok && tile_work<CG, EG>(p, unit, units, local, w); ++local) {
         const uint32_t buf = static_cast<uint32_t>(local % p.acc_bufs);
         const uint32_t acc_phase = static_cast<uint32_t>(local / p.acc_bufs) & 1;
-        const uint32_t id0 = w.half ? idesc_half[0] : idesc_full[0];
-        const uint32_t id1 = w.half ? idesc_half[1] : idesc_full[1];
+        // this work item's chunks: instruction descriptors (pairs: M = 128 for a
+        // half tile) and the offset of chunk 1's gate boxes within a K slice
+        const GroupShape gs = group_shape(p, w.eg);
+        const bool two_chunks = gs.n_chunks > 1;
+        const uint32_t m = w.half ? BLOCK_M : BLOCK_M * CG;
+        const uint32_t id0 = mma_idesc<FP8>(m, chunk_n(gs, 0));
+        const uint32_t id1 = mma_idesc<FP8>(m, two_chunks ? chunk_n(gs, 1) : N_CHUNK);
+        const uint32_t b_off1 = static_cast<uint32_t>(chunk_boxes<CG>(gs, 0) * B_BOX_BYTES);
         if (!mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + buf * p.acc_stride;
@@ -383,7 +412,7 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
                 const uint32_t accumulate = ((kb + sub) | kk) != 0;
                 const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
                 umma<FP8, kPair>(d_tmem, a_desc, gate_desc_k_slice<FP8>(b_addr, kk), id0, accumulate);
-                umma<FP8, kPair>(d_tmem + N_CHUNK, a_desc, gate_desc_k_slice<FP8>(b_addr + b_off[1], kk), id1,
+                umma<FP8, kPair>(d_tmem + N_CHUNK, a_desc, gate_desc_k_slice<FP8>(b_addr + b_off1, kk), id1,
                                  accumulate);
               }
             } else {
@@ -426,34 +455,36 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int local = 0;
     TileWork w;
-    for (; tile_work<CG>(p, unit, units, local, w); ++local) {
+    RowTopK<KMAX> top;
+    for (; tile_work<CG, EG>(p, unit, units, local, w); ++local) {
       const uint32_t buf = static_cast<uint32_t>(local % p.acc_bufs);
       const uint32_t acc_phase = static_cast<uint32_t>(local / p.acc_bufs) & 1;
       bool ok = mbar_wait(&acc_full[buf], acc_phase, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
 
-      // full tile: one row per thread, TMEM column e = expert e; half tile:
-      // per chunk c, lanes 0..63 hold experts [256c, 256c + N_c/2) and lanes
-      // 64..127 experts [256c + N_c/2, 256c + N_c) of 64 rows, in columns from 256c
+      // full tile: one row per thread, TMEM column c = expert e0 + c of the group;
+      // half tile: per chunk c, lanes 0..63 hold experts e0 + [256c, 256c + N_c/2)
+      // and lanes 64..127 experts e0 + [256c + N_c/2, 256c + N_c) of 64 rows, in
+      // columns from 256c
       const bool upper = w.half && quad >= 2;
-      RowTopK<KMAX> top;
-      top.reset();
+      if (w.eg == 0) top.reset();  // the lists run over every expert group of the tile
       const uint32_t acc_addr = lane_base + buf * p.acc_stride;
+      const GroupShape gs = group_shape(p, w.eg);
       float hs = 1.0f;  // FP8: this row's token scale
       if constexpr (FP8) {
         const int64_t my_row = w.half ? static_cast<int64_t>(w.row0) + rank * (BLOCK_M / 2) + (quad & 1) * 32 + lane
                                       : static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
         hs = my_row < p.T ? __ldg(p.hscale + my_row) : 0.0f;
       }
-      // full tiles: one pass over columns [0, E); half tiles: one per chunk
-      const int passes = w.half ? p.n_chunks : 1;
+      // full tiles: one pass over the group's columns; half tiles: one per chunk
+      const int passes = w.half ? gs.n_chunks : 1;
       for (int c = 0; c < passes; ++c) {
-        int col_base = 0, ncols = p.E;
+        int col_base = gs.e0, ncols = min(gs.n_pad, p.E - gs.e0);
         uint32_t chunk_addr = acc_addr;
         if (w.half) {
-          col_base = c * N_CHUNK + (upper ? chunk_n(p, c) / 2 : 0);
-          ncols = min(chunk_n(p, c) / 2, p.E - col_base);
+          col_base = gs.e0 + c * N_CHUNK + (upper ? chunk_n(gs, c) / 2 : 0);
+          ncols = min(chunk_n(gs, c) / 2, p.E - col_base);
           chunk_addr += static_cast<uint32_t>(c * N_CHUNK);
         }
         // 64 columns per round trip: two loads, one wait
@@ -482,11 +513,13 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           mbar_arrive(&acc_empty[buf]);
       }
 
+      if (w.eg + 1 < EG) continue;  // the tile's next expert group follows
       if (!w.half) {
         const int64_t row = static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
         if (row < p.T) top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
       } else {
-        // A half tile is a CTA's last tile, so its ring is idle: the upper lanes
+        // A half tile is a CTA's last tile (and this its last expert group), so
+        // its ring is idle: the upper lanes
         // hand their lists to the lower lanes of the same rows through it.
         const int m = (quad & 1) * 32 + lane;  // row within this CTA's 64
         float* xv = reinterpret_cast<float*>(sA) + m * KMAX;

@@ -23,7 +23,9 @@
 // More than 256 experts (up to 512): one MMA per chunk of at most 256 experts
 // and K step (chunk c in tensor-memory columns from 256c), and steps 2..5 run
 // once per 256-expert column range: each pass pushes and reduces its columns
-// and the owners keep their running top-k lists across passes.
+// and the owners keep their running top-k lists across passes.  More than 512
+// (up to 1024): steps 1..5 run once per group of 512 experts, the ring position
+// carried over; the owners' lists run over both groups.
 //
 // FP8 = true: E4M3 inputs as in the row-tile kernel (kind::f8f6f4, K-major
 // expert-major gate, 128 K values per slice); owners scale the summed logits
@@ -52,13 +54,13 @@ constexpr int PUSH_SCRATCH_BYTES = 32 * PUSH_SCRATCH_STRIDE * 4;   // one 32 x 3
 
 struct SplitHParams {
   int32_t T, H, E, k;
-  int32_t n_pad;        // total MMA N (E rounded up to 16, <= 512)
-  int32_t n_chunks;     // ceil(n_pad / 256): MMAs per K step, and exchange passes
+  int32_t n_pad;        // total MMA N (E rounded up to 16, <= 1024)
+  int32_t e_groups;     // expert groups of at most 512 (1 or 2), computed one after the other
   int32_t kps;          // K slices per ring stage (2, or 1 when n_pad > 256)
   int32_t num_tiles;    // 128-token tiles
   int32_t k_blocks;     // ceil(H / 64)
   int32_t stages;
-  int32_t b_boxes;
+  int32_t b_boxes;      // gate boxes per K slice in the ring (group 0's count, the largest)
   int32_t row_stride;   // floats per staged partial row (round_up(min(E, 256), 32) + 4)
   uint32_t tmem_cols;
   uint64_t timeout_ns;
@@ -116,106 +118,9 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer: this CTA's H slice of one tile ----------------
-      const uint64_t pol_x = l2_policy_evict_first();
-      const uint64_t pol_w = l2_policy_evict_last();
-      const uint32_t slice_tx = A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES;
-      uint32_t stage = 0, phase = 0;
-      int issued = 0;
-      for (int kb = kb0; kb < kb1; kb += p.kps) {
-        // a stage holds up to kps slices, never past this CTA's H slice
-        const int n_sub = min(p.kps, kb1 - kb);
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER, p.err_word)) break;
-        mbar_arrive_expect_tx(&full[stage], n_sub * slice_tx);
-        for (int sub = 0; sub < n_sub; ++sub) {
-          const int slot = stage * p.kps + sub;
-          const int k0 = (kb + sub) * slice_k<FP8>();
-          tma_load_2d(sA + slot * A_STAGE_BYTES, &map_x, &full[stage], k0, tile * BLOCK_M, pol_x);
-          // gate box coordinates: bf16 [H, E] map (x = expert, y = K), FP8 [E, H] map (x = K, y = expert)
-          for (int j = 0; j < p.b_boxes; ++j)
-            tma_load_2d(sB + (slot * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[stage], FP8 ? k0 : j * B_BOX_N,
-                        FP8 ? j * B_BOX_N : k0, pol_w);
-        }
-        ++issued;
-        if (++stage == static_cast<uint32_t>(p.stages)) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      const int pending = issued < p.stages ? issued : p.stages;
-      for (int n = 0; n < pending; ++n) {
-        if (stage == 0) {
-          stage = p.stages - 1;
-          phase ^= 1;
-        } else {
-          --stage;
-        }
-        mbar_wait(&full[stage], phase, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      // chunk c: N = min(256, n_pad - 256c); its gate boxes start at box 4c
-      const uint32_t idesc0 = mma_idesc<FP8>(BLOCK_M, min(p.n_pad, 256));
-      const uint32_t idesc1 = mma_idesc<FP8>(BLOCK_M, p.n_pad > 256 ? p.n_pad - 256 : 256);
-      const bool two_chunks = p.n_chunks > 1;
-      uint32_t stage = 0, phase = 0;
-      bool ok = true;
-      for (int kb = kb0; kb < kb1; kb += p.kps) {
-        const int n_sub = min(p.kps, kb1 - kb);
-        if (!mbar_wait(&full[stage], phase, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        for (int sub = 0; sub < n_sub; ++sub) {
-          const int slot = stage * p.kps + sub;
-          const uint32_t a_addr = smem_u32(sA + slot * A_STAGE_BYTES);
-          const uint32_t b_addr = smem_u32(sB + slot * p.b_boxes * B_BOX_BYTES);
-          if (two_chunks) {  // loop-invariant: no branch between the MMAs of a slice
-#pragma unroll
-            for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
-              const uint32_t accumulate = (kb + sub != kb0) | kk;
-              const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
-              umma<FP8, false>(tmem_base, a_desc, gate_desc_k_slice<FP8>(b_addr, kk), idesc0, accumulate);
-              umma<FP8, false>(tmem_base + N_CHUNK, a_desc,
-                               gate_desc_k_slice<FP8>(b_addr + (N_CHUNK / B_BOX_N) * B_BOX_BYTES, kk), idesc1,
-                               accumulate);
-            }
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
-              umma<FP8, false>(tmem_base, a_desc_k_slice(a_addr, kk), gate_desc_k_slice<FP8>(b_addr, kk), idesc0,
-                               (kb + sub != kb0) | kk);
-          }
-        }
-        umma_commit(&empty[stage]);
-        if (++stage == static_cast<uint32_t>(p.stages)) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if (ok) umma_commit(acc_full);
-      umma_commit(drain);
-      mbar_wait(drain, 0, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
-    }
-    __syncwarp();
-  }
-
-  // Epilogue warps wait for this CTA's accumulator; then all rings of the
-  // cluster are idle and may be overwritten by the exchange.
-  const bool push_warp = warp >= 2 && warp < 2 + PUSH_WARPS;
-  bool acc_ok = true;
-  if (push_warp) {
-    acc_ok = mbar_wait(acc_full, 0, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
-    acc_ok = __all_sync(0xffffffffu, acc_ok);
-  }
-
   // Owned rows: n_own <= 64 (C >= 2), and group * n_own <= SPLIT_THREADS, so one
-  // pass over the owned rows covers them all.
+  // pass over the owned rows covers them all.  The owners' lists run over every
+  // expert group.
   const int n_own = valid_rows > static_cast<int>(r) ? (valid_rows - static_cast<int>(r) + C - 1) / C : 0;
   int group = 32;  // threads per owned row: a power of two
   while (group > 1 && (n_own * group > SPLIT_THREADS || group * 8 > min(p.E, N_CHUNK))) group >>= 1;
@@ -225,102 +130,221 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
   RowTopK<KMAX> top;
   top.reset();
 
-  for (int pass = 0; pass < p.n_chunks; ++pass) {
-    const int col0 = pass * N_CHUNK;                   // first expert of this pass
-    const int pass_cols = min(N_CHUNK, p.E - col0);
-    // every ring (first pass) or every staging area (later passes) is free
-    tc_fence_before_sync();
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    tc_fence_after_sync();
+  // ring position of the producer (warp 0) and of the MMA issuer (warp 1),
+  // carried from one expert group to the next
+  uint32_t ring_stage = 0, ring_phase = 0;
 
-    // ---------------- push partial rows to their owners ----------------
-    // Each 32-row x 32-column chunk (row per thread from tensor memory) is
-    // transposed through this warp's scratch so that every remote store writes 128
-    // contiguous bytes of one row: 8 lanes per row, 4 rows per store instruction.
-    if (push_warp) {
-      const int quad = warp & 3;
-      if (acc_ok && quad * 32 < valid_rows) {
-        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
-        float* my_scratch = scratch + (warp - 2) * (PUSH_SCRATCH_BYTES / 4);
-        const int sub_row = lane >> 3;       // 0..3: row within a group of 4
-        const int col4 = (lane & 7) * 4;     // column offset within the chunk
-        // 64 columns per tensor-memory round trip, pushed as two 32-column chunks
-        for (int c0 = 0; c0 < pass_cols; c0 += 64) {
-          uint32_t v[2][32];
-          const bool second = c0 + 32 < pass_cols;  // warp-uniform
-          tmem_ld_32(lane_base + c0, v[0]);
-          if (second) tmem_ld_32(lane_base + c0 + 32, v[1]);
-          tmem_ld_wait();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (h == 1 && !second) break;
-            const int cc = c0 + 32 * h;
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(my_scratch + lane * PUSH_SCRATCH_STRIDE + j) =
-                  make_float4(__uint_as_float(v[h][j]), __uint_as_float(v[h][j + 1]), __uint_as_float(v[h][j + 2]),
-                              __uint_as_float(v[h][j + 3]));
-            __syncwarp();
-#pragma unroll
-            for (int rr = 0; rr < 32; rr += 4) {
-              const int t = quad * 32 + rr + sub_row;  // tile-local row
-              if (t < valid_rows && cc + col4 < pass_cols) {
-                const float4 val =
-                    *reinterpret_cast<const float4*>(my_scratch + (rr + sub_row) * PUSH_SCRATCH_STRIDE + col4);
-                float* dst =
-                    staging + static_cast<size_t>((t / C) * C + static_cast<int>(r)) * p.row_stride + cc + col4;
-                const unsigned owner = static_cast<unsigned>(t % C);
-                float* target = owner == r ? dst : static_cast<float*>(__cluster_map_shared_rank(dst, owner));
-                *reinterpret_cast<float4*>(target) = val;
-              }
+  for (int eg = 0; eg < p.e_groups; ++eg) {
+    // expert group eg: experts [512 eg, 512 eg + np), np = its MMA N, in chunks of 256
+    const int e0 = eg * E_GROUP;
+    const int np = eg == 0 ? min(p.n_pad, E_GROUP) : p.n_pad - E_GROUP;
+    const int n_chunks = (np + N_CHUNK - 1) / N_CHUNK;
+    const int boxes = (np + B_BOX_N - 1) / B_BOX_N;
+    const uint32_t parity = static_cast<uint32_t>(eg) & 1;
+
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---------------- TMA producer: this CTA's H slice of one tile ----------------
+        const uint64_t pol_x = l2_policy_evict_first();
+        const uint64_t pol_w = l2_policy_evict_last();
+        const uint32_t slice_tx = A_STAGE_BYTES + boxes * B_BOX_BYTES;
+        int issued = 0;
+        for (int kb = kb0; kb < kb1; kb += p.kps) {
+          // a stage holds up to kps slices, never past this CTA's H slice
+          const int n_sub = min(p.kps, kb1 - kb);
+          if (!mbar_wait(&empty[ring_stage], ring_phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER,
+                         p.err_word))
+            break;
+          mbar_arrive_expect_tx(&full[ring_stage], n_sub * slice_tx);
+          for (int sub = 0; sub < n_sub; ++sub) {
+            const int slot_i = ring_stage * p.kps + sub;
+            const int k0 = (kb + sub) * slice_k<FP8>();
+            tma_load_2d(sA + slot_i * A_STAGE_BYTES, &map_x, &full[ring_stage], k0, tile * BLOCK_M, pol_x);
+            // gate box coordinates: bf16 [H, E] map (x = expert, y = K), FP8 [E, H] map (x = K, y = expert)
+            for (int j = 0; j < boxes; ++j) {
+              const int col = e0 + j * B_BOX_N;
+              tma_load_2d(sB + (slot_i * p.b_boxes + j) * B_BOX_BYTES, &map_w, &full[ring_stage], FP8 ? k0 : col,
+                          FP8 ? col : k0, pol_w);
             }
-            __syncwarp();
+          }
+          ++issued;
+          if (++ring_stage == static_cast<uint32_t>(p.stages)) {
+            ring_stage = 0;
+            ring_phase ^= 1;
+          }
+        }
+        // every load of this group lands before the ring is reused for the exchange
+        uint32_t ds = ring_stage, dph = ring_phase;
+        const int pending = issued < p.stages ? issued : p.stages;
+        for (int n = 0; n < pending; ++n) {
+          if (ds == 0) {
+            ds = p.stages - 1;
+            dph ^= 1;
+          } else {
+            --ds;
+          }
+          mbar_wait(&full[ds], dph, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---------------- MMA issuer ----------------
+        // chunk c of the group: N = min(256, np - 256c); its gate boxes start at box 4c
+        const uint32_t idesc0 = mma_idesc<FP8>(BLOCK_M, min(np, N_CHUNK));
+        const uint32_t idesc1 = mma_idesc<FP8>(BLOCK_M, np > N_CHUNK ? np - N_CHUNK : N_CHUNK);
+        const bool two_chunks = n_chunks > 1;
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; kb += p.kps) {
+          const int n_sub = min(p.kps, kb1 - kb);
+          if (!mbar_wait(&full[ring_stage], ring_phase, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          for (int sub = 0; sub < n_sub; ++sub) {
+            const int slot_i = ring_stage * p.kps + sub;
+            const uint32_t a_addr = smem_u32(sA + slot_i * A_STAGE_BYTES);
+            const uint32_t b_addr = smem_u32(sB + slot_i * p.b_boxes * B_BOX_BYTES);
+            if (two_chunks) {  // loop-invariant: no branch between the MMAs of a slice
+#pragma unroll
+              for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
+                const uint32_t accumulate = (kb + sub != kb0) | kk;
+                const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
+                umma<FP8, false>(tmem_base, a_desc, gate_desc_k_slice<FP8>(b_addr, kk), idesc0, accumulate);
+                umma<FP8, false>(tmem_base + N_CHUNK, a_desc,
+                                 gate_desc_k_slice<FP8>(b_addr + (N_CHUNK / B_BOX_N) * B_BOX_BYTES, kk), idesc1,
+                                 accumulate);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk)
+                umma<FP8, false>(tmem_base, a_desc_k_slice(a_addr, kk), gate_desc_k_slice<FP8>(b_addr, kk), idesc0,
+                                 (kb + sub != kb0) | kk);
+            }
+          }
+          umma_commit(&empty[ring_stage]);
+          if (++ring_stage == static_cast<uint32_t>(p.stages)) {
+            ring_stage = 0;
+            ring_phase ^= 1;
+          }
+        }
+        if (ok) umma_commit(acc_full);
+        umma_commit(drain);
+        mbar_wait(drain, parity, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
+      }
+      __syncwarp();
+    }
+
+    // Epilogue warps wait for this CTA's accumulator; then all rings of the
+    // cluster are idle and may be overwritten by the exchange.
+    const bool push_warp = warp >= 2 && warp < 2 + PUSH_WARPS;
+    bool acc_ok = true;
+    if (push_warp) {
+      acc_ok = mbar_wait(acc_full, parity, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
+      acc_ok = __all_sync(0xffffffffu, acc_ok);
+    }
+
+    for (int pass = 0; pass < n_chunks; ++pass) {
+      const int col0 = pass * N_CHUNK;                        // first TMEM column of this pass
+      const int pass_cols = min(N_CHUNK, p.E - (e0 + col0));  // experts e0 + col0 .. of this pass
+      // every ring (first pass) or every staging area (later passes) is free
+      tc_fence_before_sync();
+      cluster_arrive_release();
+      cluster_wait_acquire();
+      tc_fence_after_sync();
+
+      // ---------------- push partial rows to their owners ----------------
+      // Each 32-row x 32-column chunk (row per thread from tensor memory) is
+      // transposed through this warp's scratch so that every remote store writes 128
+      // contiguous bytes of one row: 8 lanes per row, 4 rows per store instruction.
+      if (push_warp) {
+        const int quad = warp & 3;
+        if (acc_ok && quad * 32 < valid_rows) {
+          const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
+          float* my_scratch = scratch + (warp - 2) * (PUSH_SCRATCH_BYTES / 4);
+          const int sub_row = lane >> 3;       // 0..3: row within a group of 4
+          const int col4 = (lane & 7) * 4;     // column offset within the chunk
+          // 64 columns per tensor-memory round trip, pushed as two 32-column chunks
+          for (int c0 = 0; c0 < pass_cols; c0 += 64) {
+            uint32_t v[2][32];
+            const bool second = c0 + 32 < pass_cols;  // warp-uniform
+            tmem_ld_32(lane_base + c0, v[0]);
+            if (second) tmem_ld_32(lane_base + c0 + 32, v[1]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (h == 1 && !second) break;
+              const int cc = c0 + 32 * h;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(my_scratch + lane * PUSH_SCRATCH_STRIDE + j) =
+                    make_float4(__uint_as_float(v[h][j]), __uint_as_float(v[h][j + 1]), __uint_as_float(v[h][j + 2]),
+                                __uint_as_float(v[h][j + 3]));
+              __syncwarp();
+#pragma unroll
+              for (int rr = 0; rr < 32; rr += 4) {
+                const int t = quad * 32 + rr + sub_row;  // tile-local row
+                if (t < valid_rows && cc + col4 < pass_cols) {
+                  const float4 val =
+                      *reinterpret_cast<const float4*>(my_scratch + (rr + sub_row) * PUSH_SCRATCH_STRIDE + col4);
+                  float* dst =
+                      staging + static_cast<size_t>((t / C) * C + static_cast<int>(r)) * p.row_stride + cc + col4;
+                  const unsigned owner = static_cast<unsigned>(t % C);
+                  float* target = owner == r ? dst : static_cast<float*>(__cluster_map_shared_rank(dst, owner));
+                  *reinterpret_cast<float4*>(target) = val;
+                }
+              }
+              __syncwarp();
+            }
           }
         }
       }
-    }
-    tc_fence_before_sync();
-    cluster_arrive_release();  // every owner's staging area is complete past this point
-    cluster_wait_acquire();
-    if (warp == 1 && pass + 1 == p.n_chunks) {  // all tensor-memory reads of this CTA are done
-      tc_fence_after_sync();
-      tmem_dealloc(tmem_base, p.tmem_cols);
-    }
+      tc_fence_before_sync();
+      cluster_arrive_release();  // every owner's staging area is complete past this point
+      cluster_wait_acquire();
+      if (warp == 1 && eg + 1 == p.e_groups && pass + 1 == n_chunks) {  // all tensor-memory reads are done
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, p.tmem_cols);
+      }
 
-    // ---------------- reduce owned rows of this pass into the running top-k ----------------
-    if (active) {
-      float hs = 1.0f;  // FP8: the row's token scale
-      if constexpr (FP8) hs = __ldg(p.hscale + static_cast<int64_t>(tile) * BLOCK_M + static_cast<int>(r) + C * slot);
-      // segment `seg` takes every group-th float4 of the row: consecutive lanes
-      // read consecutive 16-byte words (no bank conflicts), and each thread still
-      // offers its columns in increasing order
-      const float* rows = staging + static_cast<size_t>(slot) * C * p.row_stride;
-      for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
-        float4 v[C];
+      // ---------------- reduce owned rows of this pass into the running top-k ----------------
+      if (active) {
+        float hs = 1.0f;  // FP8: the row's token scale
+        if constexpr (FP8) hs = __ldg(p.hscale + static_cast<int64_t>(tile) * BLOCK_M + static_cast<int>(r) + C * slot);
+        // segment `seg` takes every group-th float4 of the row: consecutive lanes
+        // read consecutive 16-byte words (no bank conflicts), and each thread still
+        // offers its columns in increasing order
+        const float* rows = staging + static_cast<size_t>(slot) * C * p.row_stride;
+        const int ebase = e0 + col0;
+        for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
+          float4 v[C];
 #pragma unroll
-        for (int q = 0; q < C; ++q) v[q] = *reinterpret_cast<const float4*>(rows + q * p.row_stride + c);
-        float4 acc = v[0];
+          for (int q = 0; q < C; ++q) v[q] = *reinterpret_cast<const float4*>(rows + q * p.row_stride + c);
+          float4 acc = v[0];
 #pragma unroll
-        for (int q = 1; q < C; ++q) {  // rank order: the same sum whichever CTA owns the row
-          acc.x += v[q].x;
-          acc.y += v[q].y;
-          acc.z += v[q].z;
-          acc.w += v[q].w;
+          for (int q = 1; q < C; ++q) {  // rank order: the same sum whichever CTA owns the row
+            acc.x += v[q].x;
+            acc.y += v[q].y;
+            acc.z += v[q].z;
+            acc.w += v[q].w;
+          }
+          if constexpr (FP8) {  // expert scales of columns past E are never offered
+            const int e = ebase + c;
+            acc.x = acc.x * __ldg(p.gscale + min(e, p.E - 1)) * hs;
+            acc.y = acc.y * __ldg(p.gscale + min(e + 1, p.E - 1)) * hs;
+            acc.z = acc.z * __ldg(p.gscale + min(e + 2, p.E - 1)) * hs;
+            acc.w = acc.w * __ldg(p.gscale + min(e + 3, p.E - 1)) * hs;
+          }
+          top.offer(acc.x, ebase + c);
+          if (c + 1 < pass_cols) top.offer(acc.y, ebase + c + 1);
+          if (c + 2 < pass_cols) top.offer(acc.z, ebase + c + 2);
+          if (c + 3 < pass_cols) top.offer(acc.w, ebase + c + 3);
         }
-        if constexpr (FP8) {  // expert scales of columns past E are never offered
-          const int e = col0 + c;
-          acc.x = acc.x * __ldg(p.gscale + min(e, p.E - 1)) * hs;
-          acc.y = acc.y * __ldg(p.gscale + min(e + 1, p.E - 1)) * hs;
-          acc.z = acc.z * __ldg(p.gscale + min(e + 2, p.E - 1)) * hs;
-          acc.w = acc.w * __ldg(p.gscale + min(e + 3, p.E - 1)) * hs;
-        }
-        top.offer(acc.x, col0 + c);
-        if (c + 1 < pass_cols) top.offer(acc.y, col0 + c + 1);
-        if (c + 2 < pass_cols) top.offer(acc.z, col0 + c + 2);
-        if (c + 3 < pass_cols) top.offer(acc.w, col0 + c + 3);
       }
     }
+    // the next expert group's loads overwrite this CTA's staging area: every
+    // owner of this CTA has read it
+    if (eg + 1 < p.e_groups) __syncthreads();
   }
 
   // ---------------- merge the segments, softmax, store ----------------

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -49,8 +50,9 @@ constexpr int kMaxSplit = 16;  // CTAs per cluster in the split-H variant (16 ne
 // Split-H plan: one 128-token tile per cluster of C CTAs, single-CTA MMAs.
 tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* plan) {
   const int n_pad = round_up(static_cast<int>(E), 16);
-  const int kps = n_pad > tkg::N_CHUNK ? 1 : tkg::KB_PER_STAGE;  // a slice of 512 experts is 80 KB
-  const int b_boxes = (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+  const int g_pad = n_pad < tkg::E_GROUP ? n_pad : tkg::E_GROUP;  // MMA N of the (largest) expert group
+  const int kps = g_pad > tkg::N_CHUNK ? 1 : tkg::KB_PER_STAGE;   // a slice of 512 experts is 80 KB
+  const int b_boxes = (g_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES;
   const int scratch = tkg::PUSH_WARPS * tkg::PUSH_SCRATCH_BYTES;
   int stages = (kMaxDynamicSmem - kSmemReserve - scratch) / (kps * stage_bytes);
@@ -70,8 +72,9 @@ tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* p
   plan->cluster = C;
   plan->threads = tkg::SPLIT_THREADS;
   plan->smem_bytes = stages * kps * stage_bytes + scratch + kSmemReserve;
-  plan->tmem_cols = static_cast<int32_t>(pow2_at_least(round_up(n_pad, 32)));
+  plan->tmem_cols = static_cast<int32_t>(pow2_at_least(round_up(g_pad, 32)));
   plan->slices_per_stage = kps;
+  plan->expert_groups = n_pad > tkg::E_GROUP ? 2 : 1;
   return TK_OK;
 }
 
@@ -121,9 +124,10 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   const bool pair = E > 64;  // gate halves of >= 64 experts per CTA (128-byte swizzle blocks)
   const int cg = pair ? 2 : 1;
   const int n_pad = pair ? round_up(static_cast<int>(E), 128) : round_up(static_cast<int>(E), 16);
-  const int acc_stride = round_up(n_pad, 32);
+  const int g_pad = n_pad < tkg::E_GROUP ? n_pad : tkg::E_GROUP;  // MMA N of the (largest) expert group
+  const int acc_stride = round_up(g_pad, 32);
   const int acc_bufs = 2 * acc_stride <= 512 ? 2 : 1;  // 512 tensor-memory columns
-  const int b_boxes = pair ? n_pad / 2 / tkg::B_BOX_N : (n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+  const int b_boxes = pair ? g_pad / 2 / tkg::B_BOX_N : (g_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::KB_PER_STAGE * (tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES);
   int stages = (kMaxDynamicSmem - kSmemReserve) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
@@ -160,6 +164,7 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   plan->smem_bytes = stages * stage_bytes + kSmemReserve;
   plan->tmem_cols = static_cast<int32_t>(pow2_at_least(acc_bufs * acc_stride));
   plan->slices_per_stage = tkg::KB_PER_STAGE;
+  plan->expert_groups = n_pad > tkg::E_GROUP ? 2 : 1;
   return TK_OK;
 }
 
@@ -235,8 +240,9 @@ bool set_smem_limit(Kernel kernel) {
 
 template <int KMAX, bool FP8>
 bool set_up_kernels_of() {
-  bool ok = set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 1, FP8>) &&
-            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2, FP8>) &&
+  bool ok = set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 1, FP8, 1>) &&
+            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2, FP8, 1>) &&
+            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2, FP8, 2>) &&
             set_smem_limit(tkg::gating_split_h_kernel<KMAX, 2, FP8>) &&
             set_smem_limit(tkg::gating_split_h_kernel<KMAX, 4, FP8>) &&
             set_smem_limit(tkg::gating_split_h_kernel<KMAX, 8, FP8>) &&
@@ -317,10 +323,10 @@ const DeviceState* device_state() {
   return &d;
 }
 
-template <int KMAX, int CG, bool FP8>
+template <int KMAX, int CG, bool FP8, int EG>
 tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
                            const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
-  auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG, FP8>;
+  auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG, FP8, EG>;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
@@ -374,8 +380,11 @@ tk_status launch_split_h(const tk_gating_plan& plan, int max_cluster, const CUte
 template <int KMAX, bool FP8>
 tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
                              const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
-  if (pl.variant == TK_VARIANT_ROW_PAIRS) return launch_row_tiles<KMAX, 2, FP8>(pl, mx, mx64, mw, prm, stream);
-  return launch_row_tiles<KMAX, 1, FP8>(pl, mx, mx64, mw, prm, stream);
+  if (pl.variant == TK_VARIANT_ROW_PAIRS) {
+    if (pl.expert_groups == 2) return launch_row_tiles<KMAX, 2, FP8, 2>(pl, mx, mx64, mw, prm, stream);
+    return launch_row_tiles<KMAX, 2, FP8, 1>(pl, mx, mx64, mw, prm, stream);
+  }
+  return launch_row_tiles<KMAX, 1, FP8, 1>(pl, mx, mx64, mw, prm, stream);
 }
 
 // Launch the planned kernel on encoded maps.  FP8: hscale / gscale are the
@@ -392,12 +401,12 @@ tk_status launch_planned(const tk_gating_plan& pl, const DeviceState* dev, const
     sp.E = static_cast<int32_t>(E);
     sp.k = k;
     sp.n_pad = pl.n_pad;
-    sp.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
+    sp.e_groups = pl.expert_groups;
     sp.kps = pl.slices_per_stage;
     sp.num_tiles = pl.num_tiles;
     sp.k_blocks = pl.k_blocks;
     sp.stages = pl.stages;
-    sp.b_boxes = (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+    sp.b_boxes = (std::min(pl.n_pad, tkg::E_GROUP) + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
     sp.row_stride = split_row_stride(E);
     sp.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
     sp.timeout_ns = g_timeout_ns;
@@ -421,15 +430,15 @@ tk_status launch_planned(const tk_gating_plan& pl, const DeviceState* dev, const
   prm.E = static_cast<int32_t>(E);
   prm.k = k;
   prm.n_pad = pl.n_pad;
-  prm.n_chunks = (pl.n_pad + tkg::N_CHUNK - 1) / tkg::N_CHUNK;
-  prm.acc_stride = round_up(pl.n_pad, 32);
+  prm.e_groups = pl.expert_groups;
+  prm.acc_stride = round_up(std::min(pl.n_pad, tkg::E_GROUP), 32);
   prm.acc_bufs = 2 * prm.acc_stride <= 512 ? 2 : 1;
   prm.num_tiles = pl.num_tiles;
   prm.num_half = pl.num_half_tiles;
   prm.k_blocks = pl.k_blocks;
   prm.stages = pl.stages;
-  prm.b_boxes = pl.variant == TK_VARIANT_ROW_PAIRS ? pl.n_pad / 2 / tkg::B_BOX_N
-                                                   : (pl.n_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
+  const int g_pad = std::min(pl.n_pad, tkg::E_GROUP);
+  prm.b_boxes = pl.variant == TK_VARIANT_ROW_PAIRS ? g_pad / 2 / tkg::B_BOX_N : (g_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   prm.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
   prm.timeout_ns = g_timeout_ns;
   prm.scores = scores;

@@ -45,7 +45,7 @@ def test_status_strings():
     ((8, 60, 16, 2), tk.TK_ERR_UNSUPPORTED),        # H % 8
     ((8, 64, 20, 2), tk.TK_ERR_UNSUPPORTED),        # E % 8
     ((8, 64, 8, 2), tk.TK_ERR_UNSUPPORTED),         # E < 16
-    ((8, 64, 520, 2), tk.TK_ERR_UNSUPPORTED),       # E > 512
+    ((8, 64, 1032, 2), tk.TK_ERR_UNSUPPORTED),      # E > 1024
     ((8, 64, 64, 33), tk.TK_ERR_UNSUPPORTED),       # k > 32
 ])
 def test_invalid_sizes_rejected_before_cuda(args, code):
@@ -87,7 +87,7 @@ def test_plans_for_router_workloads():
         if p["variant"] == 1:
             assert p["grid"] == min(p["num_tiles"], 148) and p["cluster"] == 1
         if p["variant"] == 3:
-            assert p["cluster"] == 2 and p["block_m"] == 256 and p["n_pad"] in (128, 256, 384, 512)
+            assert p["cluster"] == 2 and p["block_m"] == 256 and p["n_pad"] % 128 == 0 and p["n_pad"] <= 1024
             assert p["grid"] == 2 * min(p["num_tiles"], 74)
         if p["variant"] == 2:
             C = p["cluster"]
@@ -123,9 +123,10 @@ def test_plan_variant_choice():
 
 def test_plan_tmem_and_smem_budget():
     for T in (1, 1000, 30000):
-        for E in range(16, 513, 8):
+        for E in range(16, 1025, 8):
             p = tk.make_plan(T, 7168, E, min(8, E), 148)
-            acc = (p["n_pad"] + 31) // 32 * 32
+            assert p["expert_groups"] == (2 if p["n_pad"] > 512 else 1)
+            acc = (min(p["n_pad"], 512) + 31) // 32 * 32
             # split-H keeps one accumulator; row tiles two, or one when two do not fit
             buffers = 1 if p["variant"] == 2 or 2 * acc > 512 else 2
             assert p["tmem_cols"] >= buffers * acc
@@ -148,13 +149,17 @@ def test_plan_large_expert_counts():
     assert p["variant"] == 2 and p["slices_per_stage"] == 1 and p["tmem_cols"] == 512
     p = tk.make_plan(4096, 7168, 256, 8, 148)
     assert p["slices_per_stage"] == 2
+    p = tk.make_plan(65536, 7168, 1024, 8, 148)     # two expert groups of 512, one after the other
+    assert p["variant"] == 3 and p["n_pad"] == 1024 and p["expert_groups"] == 2 and p["tmem_cols"] == 512
+    p = tk.make_plan(1, 7168, 1000, 8, 148)
+    assert p["variant"] == 2 and p["expert_groups"] == 2 and p["tmem_cols"] == 512
 
 
 def test_fp8_entry_point_rejects_before_cuda():
     f = tk.fused_topk_gating_fp8_ptr
     assert f(16, 16, 16, 16, 8, 72, 16, 2, 16, 16) == tk.TK_ERR_UNSUPPORTED        # H % 16 != 0
     assert f(16, 16, 16, 16, 8, 64, 16, 17, 16, 16) == tk.TK_ERR_INVALID_ARG       # k > E
-    assert f(16, 16, 16, 16, 8, 64, 520, 2, 16, 16) == tk.TK_ERR_UNSUPPORTED       # E > 512
+    assert f(16, 16, 16, 16, 8, 64, 1032, 2, 16, 16) == tk.TK_ERR_UNSUPPORTED      # E > 1024
     assert f(16, 0, 16, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_INVALID_ARG         # null scale
     assert f(16, 20, 16, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_ALIGNMENT          # scale not 16-byte aligned
     assert f(0, 0, 0, 0, 0, 64, 16, 2, 0, 0) == tk.TK_OK                             # T == 0

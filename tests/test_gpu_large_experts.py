@@ -31,6 +31,8 @@ def clean_error_word():
     (129, 512, 264, 1), (300, 520, 504, 17),
     # CTA pairs, two chunks, single accumulator (and half tiles: T just above a full round)
     (20000, 512, 512, 8), (30000, 512, 320, 32), (19999, 256, 448, 5), (40000, 128, 264, 3),
+    # two expert groups of up to 512 (E up to 1024), split-H and pairs
+    (1, 7168, 1024, 8), (100, 1024, 640, 32), (4096, 512, 1024, 8), (20000, 256, 1024, 8), (30000, 256, 776, 16),
     # k up to 32 with one chunk
     (2000, 1024, 256, 32), (40000, 512, 256, 32), (5000, 256, 64, 32), (700, 256, 32, 32),
 ])
@@ -53,6 +55,20 @@ def test_ties_across_chunk_and_half_boundaries(T):
         w[:, a] = workloads.round_bf16(workloads.bf16_to_f64(w[:, a]) * 3.0)
         w[:, b] = w[:, a]
     check_against_oracle(wl.hidden(), w, k, duplicate_pairs=pairs, label=f"ties_{T}")
+
+
+@pytest.mark.parametrize("T", [300, 24000])
+def test_ties_across_expert_groups(T):
+    # experts 511 and 512 sit in different groups (computed one after the other):
+    # equal logits must still go to the lower index
+    E, H, k = 1024, 256, 8
+    wl = workloads.RouterWorkload(f"gties_{T}", T, H, E, k, seed=17)
+    w = wl.gate_weight().copy()
+    pairs = ((511, 512), (0, 1023), (300, 700), (255, 256))
+    for a, b in pairs:
+        w[:, a] = workloads.round_bf16(workloads.bf16_to_f64(w[:, a]) * 3.0)
+        w[:, b] = w[:, a]
+    check_against_oracle(wl.hidden(), w, k, duplicate_pairs=pairs, label=f"gties_{T}")
 
 
 def test_large_e_workload_sampled_rows():

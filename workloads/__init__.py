@@ -175,8 +175,9 @@ DECODE = tuple(RouterWorkload(f"decode_T{t}", t, 7168, 256, 8) for t in DECODE_T
 # chunks of 256 experts, top-32 selection.
 LARGE_E = RouterWorkload("large_e", 65536, 7168, 512, 8)
 LARGE_K = RouterWorkload("large_k", 4096, 7168, 512, 32)
+E1024 = RouterWorkload("e1024", 65536, 7168, 1024, 8)  # two expert groups of 512
 
-WORKLOADS = {w.name: w for w in (TINY, DEEPSEEK, SKEW, TRAIN, LARGE_E, LARGE_K) + DECODE}
+WORKLOADS = {w.name: w for w in (TINY, DEEPSEEK, SKEW, TRAIN, LARGE_E, LARGE_K, E1024) + DECODE}
 
 
 def quantize_e4m3_rows(values: np.ndarray):
