@@ -23,10 +23,10 @@ LIB = os.path.join(PKG, "libtk_gating.so")
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
-    "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+    "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "--expt-relaxed-constexpr",
-    "-cudart", "static",
 ]
+LINK_FLAGS = ["-shared", "-cudart", "static", "-gencode", "arch=compute_100a,code=sm_100a"]
 
 
 def nvcc() -> str:
@@ -76,14 +76,34 @@ def is_stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every csrc/*.cu to an object in parallel (the bf16 and FP8 kernel
+    instances live in separate translation units), then link the library."""
     if not force and not is_stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    objdir = os.path.join(PKG, f"_build_{os.getpid()}")
+    os.makedirs(objdir, exist_ok=True)
+    try:
+        procs = []
+        for src in sources():
+            obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
+            cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+            if verbose:
+                cmd.insert(1, "-Xptxas=-v")
+            procs.append((src, obj, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
+        failed = []
+        for src, _, proc in procs:
+            out, _ = proc.communicate()
+            if out:
+                sys.stdout.write(out)
+            if proc.returncode != 0:
+                failed.append(os.path.basename(src))
+        if failed:
+            raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(failed)})")
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([nvcc(), *LINK_FLAGS, *[obj for _, obj, _ in procs], "-o", tmp])
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(objdir, ignore_errors=True)
     return LIB
 
 

@@ -1,0 +1,57 @@
+// Launch interface of the fused gating kernels, shared by the host entry points
+// (tk_gating.cu) and the two translation units that instantiate the kernels
+// (gating_bf16.cu, gating_fp8.cu; the definitions are in gating_launch_impl.cuh).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tk_gating.h"
+#include "gating_row_tiles.cuh"
+#include "gating_split_h.cuh"
+
+namespace tkg {
+
+constexpr int kMaxDynamicSmem = 232448;  // 227 KB opt-in per CTA on sm_100
+
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// Floats per staged partial row of the split-H exchange (one pass of up to 256
+// experts; +4 spreads the rows over the shared-memory banks).
+inline int split_row_stride(int64_t E) { return round_up(static_cast<int>(E < N_CHUNK ? E : N_CHUNK), 32) + 4; }
+
+// What a launch needs from the device state.
+struct LaunchEnv {
+  int max_split_cluster;  // largest split-H cluster the device co-schedules
+  uint32_t* err_word;     // device error word of the bounded waits
+  uint64_t timeout_ns;    // bounded-wait limit
+};
+
+// Shared-memory limits (and non-portable cluster sizes) of every kernel instance
+// of one precision; once per device.
+template <bool FP8>
+bool set_up_gating_kernels();
+
+// Launch the planned kernel on encoded maps.  FP8: hscale / gscale are the
+// per-token and per-expert scales (unused for bf16).
+template <bool FP8>
+tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const CUtensorMap& mx,
+                         const CUtensorMap& mx64, const CUtensorMap& mw, int64_t T, int64_t H, int64_t E, int32_t k,
+                         float* scores, int32_t* ids, const float* hscale, const float* gscale, cudaStream_t stream);
+
+extern template bool set_up_gating_kernels<false>();
+extern template bool set_up_gating_kernels<true>();
+extern template tk_status launch_planned<false>(const tk_gating_plan&, const LaunchEnv&, const CUtensorMap&,
+                                                const CUtensorMap&, const CUtensorMap&, int64_t, int64_t, int64_t,
+                                                int32_t, float*, int32_t*, const float*, const float*, cudaStream_t);
+extern template tk_status launch_planned<true>(const tk_gating_plan&, const LaunchEnv&, const CUtensorMap&,
+                                               const CUtensorMap&, const CUtensorMap&, int64_t, int64_t, int64_t,
+                                               int32_t, float*, int32_t*, const float*, const float*, cudaStream_t);
+
+// Clusters of 2, 4, 8 and 16 full-shared-memory split-H CTAs that the current
+// device runs at once, into counts[0..3] (0 where a size cannot run).
+void measure_split_cluster_capacity(int counts[4]);
+
+}  // namespace tkg

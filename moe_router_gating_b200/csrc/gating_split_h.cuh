@@ -316,7 +316,8 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
         // offers its columns in increasing order
         const float* rows = staging + static_cast<size_t>(slot) * C * p.row_stride;
         const int ebase = e0 + col0;
-        for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
+        // the summed (and, FP8, scaled) logits of columns c .. c+3 of this row
+        auto column_quad = [&](int c) {
           float4 v[C];
 #pragma unroll
           for (int q = 0; q < C; ++q) v[q] = *reinterpret_cast<const float4*>(rows + q * p.row_stride + c);
@@ -335,6 +336,10 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
             acc.z = acc.z * __ldg(p.gscale + min(e + 2, p.E - 1)) * hs;
             acc.w = acc.w * __ldg(p.gscale + min(e + 3, p.E - 1)) * hs;
           }
+          return acc;
+        };
+        for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
+          const float4 acc = column_quad(c);
           top.offer(acc.x, ebase + c);
           if (c + 1 < pass_cols) top.offer(acc.y, ebase + c + 1);
           if (c + 2 < pass_cols) top.offer(acc.z, ebase + c + 2);

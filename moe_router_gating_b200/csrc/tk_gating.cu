@@ -1,6 +1,7 @@
 // C ABI of the fused MoE top-k gating library (declared in include/tk_gating.h):
-// argument validation, launch planning, TMA descriptor encoding and launches.
-// The computation itself is in the kernels included below.
+// argument validation, launch planning, TMA descriptor encoding and the calls
+// into the launch code, which gating_bf16.cu and gating_fp8.cu instantiate
+// (two translation units, compiled in parallel).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -10,8 +11,7 @@
 #include <mutex>
 
 #include "tk_gating.h"
-#include "gating_row_tiles.cuh"
-#include "gating_split_h.cuh"
+#include "gating_launch.cuh"
 
 namespace {
 
@@ -19,13 +19,13 @@ __device__ uint32_t g_tk_error_word = 0;
 
 uint64_t g_timeout_ns = 1000000000ull;  // bounded-wait limit for kernels launched from here
 
-constexpr int kMaxDynamicSmem = 232448;  // 227 KB opt-in per CTA on sm_100
+constexpr int kMaxDynamicSmem = tkg::kMaxDynamicSmem;
 constexpr int kSmemReserve = 1024 + 256;  // 1 KB alignment pad + barriers and flags
 constexpr int kMaxStages = 8;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int round_up(int v, int m) { return (v + m - 1) / m * m; }
+using tkg::round_up;
 
 uint32_t pow2_at_least(uint32_t v) {
   uint32_t c = 32;
@@ -41,9 +41,7 @@ tk_status validate_sizes(int64_t T, int64_t H, int64_t E, int32_t k) {
   return TK_OK;
 }
 
-// Floats per staged partial row of the split-H exchange (one pass of up to 256
-// experts; +4 spreads the rows over the shared-memory banks).
-int split_row_stride(int64_t E) { return round_up(static_cast<int>(E < tkg::N_CHUNK ? E : tkg::N_CHUNK), 32) + 4; }
+using tkg::split_row_stride;
 
 constexpr int kMaxSplit = 16;  // CTAs per cluster in the split-H variant (16 needs non-portable clusters)
 
@@ -233,59 +231,6 @@ constexpr int kMaxDevices = 64;
 DeviceState g_devices[kMaxDevices];
 std::mutex g_devices_mutex;
 
-template <typename Kernel>
-bool set_smem_limit(Kernel kernel) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem) == cudaSuccess;
-}
-
-template <int KMAX, bool FP8>
-bool set_up_kernels_of() {
-  bool ok = set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 1, FP8, 1>) &&
-            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2, FP8, 1>) &&
-            set_smem_limit(tkg::gating_row_tiles_kernel<KMAX, 2, FP8, 2>) &&
-            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 2, FP8>) &&
-            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 4, FP8>) &&
-            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 8, FP8>) &&
-            set_smem_limit(tkg::gating_split_h_kernel<KMAX, 16, FP8>);
-  return ok && cudaFuncSetAttribute(tkg::gating_split_h_kernel<KMAX, 16, FP8>,
-                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
-}
-
-template <int KMAX>
-bool set_up_kernels() {
-  return set_up_kernels_of<KMAX, false>() && set_up_kernels_of<KMAX, true>();
-}
-
-// Clusters of each size 2^i (i = 1..4) of full-shared-memory CTAs that the
-// device runs at once.
-ClusterCapacity measure_cluster_capacity(int num_sms) {
-  ClusterCapacity cap;
-  cap.n[0] = num_sms;
-  for (int i = 1; i <= 4; ++i) {
-    const int C = 1 << i;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C);
-    cfg.blockDim = dim3(tkg::SPLIT_THREADS);
-    cfg.dynamicSmemBytes = kMaxDynamicSmem;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    cudaError_t e = C == 16 ? cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 16, false>, &cfg)
-                            : cudaOccupancyMaxActiveClusters(&n, tkg::gating_split_h_kernel<8, 8, false>, &cfg);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      n = 0;
-    }
-    cap.n[i] = n;
-  }
-  return cap;
-}
-
 const DeviceState* device_state() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -305,13 +250,14 @@ const DeviceState* device_state() {
     return &d;
   }
   void* err = nullptr;
-  if (cudaGetSymbolAddress(&err, g_tk_error_word) != cudaSuccess || !set_up_kernels<1>() || !set_up_kernels<2>() ||
-      !set_up_kernels<4>() || !set_up_kernels<8>() || !set_up_kernels<16>() || !set_up_kernels<32>()) {
+  if (cudaGetSymbolAddress(&err, g_tk_error_word) != cudaSuccess || !tkg::set_up_gating_kernels<false>() ||
+      !tkg::set_up_gating_kernels<true>()) {
     cudaGetLastError();
     return nullptr;  // not cached: a later call retries
   }
   d.err_word = static_cast<uint32_t*>(err);
-  d.capacity = measure_cluster_capacity(d.num_sms);
+  d.capacity.n[0] = d.num_sms;
+  tkg::measure_split_cluster_capacity(d.capacity.n + 1);
   d.max_split_cluster = 0;
   for (int i = 4; i >= 1; --i)
     if (d.capacity.n[i] > 0) {
@@ -321,138 +267,6 @@ const DeviceState* device_state() {
   d.status = TK_OK;
   d.ready = true;
   return &d;
-}
-
-template <int KMAX, int CG, bool FP8, int EG>
-tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
-                           const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
-  auto kernel = tkg::gating_row_tiles_kernel<KMAX, CG, FP8, EG>;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CG;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.grid);
-  cfg.blockDim = dim3(pl.threads);
-  cfg.dynamicSmemBytes = pl.smem_bytes;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = CG > 1 ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, kernel, mx, mx64, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
-  return TK_OK;
-}
-
-template <int KMAX, int C, bool FP8>
-tk_status launch_split_h_c(const tk_gating_plan& plan, const CUtensorMap& mx, const CUtensorMap& mw,
-                           const tkg::SplitHParams& prm, cudaStream_t stream) {
-  auto kernel = tkg::gating_split_h_kernel<KMAX, C, FP8>;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.num_tiles * C);
-  cfg.blockDim = dim3(plan.threads);
-  cfg.dynamicSmemBytes = plan.smem_bytes;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, mx, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
-  return TK_OK;
-}
-
-template <int KMAX, bool FP8>
-tk_status launch_split_h(const tk_gating_plan& plan, int max_cluster, const CUtensorMap& mx, const CUtensorMap& mw,
-                         const tkg::SplitHParams& prm, cudaStream_t stream) {
-  int C = plan.cluster;
-  while (C > max_cluster) C >>= 1;  // the largest cluster the device co-schedules
-  switch (C) {
-    case 16: return launch_split_h_c<KMAX, 16, FP8>(plan, mx, mw, prm, stream);
-    case 8: return launch_split_h_c<KMAX, 8, FP8>(plan, mx, mw, prm, stream);
-    case 4: return launch_split_h_c<KMAX, 4, FP8>(plan, mx, mw, prm, stream);
-    case 2: return launch_split_h_c<KMAX, 2, FP8>(plan, mx, mw, prm, stream);
-    default: return TK_ERR_UNSUPPORTED;
-  }
-}
-
-template <int KMAX, bool FP8>
-tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
-                             const CUtensorMap& mw, const tkg::RowTileParams& prm, cudaStream_t stream) {
-  if (pl.variant == TK_VARIANT_ROW_PAIRS) {
-    if (pl.expert_groups == 2) return launch_row_tiles<KMAX, 2, FP8, 2>(pl, mx, mx64, mw, prm, stream);
-    return launch_row_tiles<KMAX, 2, FP8, 1>(pl, mx, mx64, mw, prm, stream);
-  }
-  return launch_row_tiles<KMAX, 1, FP8, 1>(pl, mx, mx64, mw, prm, stream);
-}
-
-// Launch the planned kernel on encoded maps.  FP8: hscale / gscale are the
-// per-token and per-expert scales (unused for bf16).
-template <bool FP8>
-tk_status launch_planned(const tk_gating_plan& pl, const DeviceState* dev, const CUtensorMap& mx,
-                         const CUtensorMap& mx64, const CUtensorMap& mw, int64_t T, int64_t H, int64_t E, int32_t k,
-                         float* scores, int32_t* ids, const float* hscale, const float* gscale, cudaStream_t stream) {
-  uint32_t* err = dev->err_word;
-  if (pl.variant == TK_VARIANT_SPLIT_H) {
-    tkg::SplitHParams sp;
-    sp.T = static_cast<int32_t>(T);
-    sp.H = static_cast<int32_t>(H);
-    sp.E = static_cast<int32_t>(E);
-    sp.k = k;
-    sp.n_pad = pl.n_pad;
-    sp.e_groups = pl.expert_groups;
-    sp.kps = pl.slices_per_stage;
-    sp.num_tiles = pl.num_tiles;
-    sp.k_blocks = pl.k_blocks;
-    sp.stages = pl.stages;
-    sp.b_boxes = (std::min(pl.n_pad, tkg::E_GROUP) + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
-    sp.row_stride = split_row_stride(E);
-    sp.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
-    sp.timeout_ns = g_timeout_ns;
-    sp.scores = scores;
-    sp.ids = ids;
-    sp.err_word = err;
-    sp.hscale = hscale;
-    sp.gscale = gscale;
-    const int mc = dev->max_split_cluster;
-    if (k <= 1) return launch_split_h<1, FP8>(pl, mc, mx, mw, sp, stream);
-    if (k <= 2) return launch_split_h<2, FP8>(pl, mc, mx, mw, sp, stream);
-    if (k <= 4) return launch_split_h<4, FP8>(pl, mc, mx, mw, sp, stream);
-    if (k <= 8) return launch_split_h<8, FP8>(pl, mc, mx, mw, sp, stream);
-    if (k <= 16) return launch_split_h<16, FP8>(pl, mc, mx, mw, sp, stream);
-    return launch_split_h<32, FP8>(pl, mc, mx, mw, sp, stream);
-  }
-
-  tkg::RowTileParams prm;
-  prm.T = static_cast<int32_t>(T);
-  prm.H = static_cast<int32_t>(H);
-  prm.E = static_cast<int32_t>(E);
-  prm.k = k;
-  prm.n_pad = pl.n_pad;
-  prm.e_groups = pl.expert_groups;
-  prm.acc_stride = round_up(std::min(pl.n_pad, tkg::E_GROUP), 32);
-  prm.acc_bufs = 2 * prm.acc_stride <= 512 ? 2 : 1;
-  prm.num_tiles = pl.num_tiles;
-  prm.num_half = pl.num_half_tiles;
-  prm.k_blocks = pl.k_blocks;
-  prm.stages = pl.stages;
-  const int g_pad = std::min(pl.n_pad, tkg::E_GROUP);
-  prm.b_boxes = pl.variant == TK_VARIANT_ROW_PAIRS ? g_pad / 2 / tkg::B_BOX_N : (g_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
-  prm.tmem_cols = static_cast<uint32_t>(pl.tmem_cols);
-  prm.timeout_ns = g_timeout_ns;
-  prm.scores = scores;
-  prm.ids = ids;
-  prm.err_word = err;
-  prm.hscale = hscale;
-  prm.gscale = gscale;
-
-  if (k <= 1) return launch_row_variant<1, FP8>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 2) return launch_row_variant<2, FP8>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 4) return launch_row_variant<4, FP8>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 8) return launch_row_variant<8, FP8>(pl, mx, mx64, mw, prm, stream);
-  if (k <= 16) return launch_row_variant<16, FP8>(pl, mx, mx64, mw, prm, stream);
-  return launch_row_variant<32, FP8>(pl, mx, mx64, mw, prm, stream);
 }
 
 tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int64_t H, int64_t E, int32_t k,
@@ -477,7 +291,8 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
                                                 tkg::BLOCK_K, tkg::BLOCK_M / 2)) ||
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
-  return launch_planned<false>(pl, dev, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, stream);
+  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns};
+  return tkg::launch_planned<false>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, stream);
 }
 
 // FP8 sizes: H a multiple of 16 (16-byte rows of 8-bit values); E and k as bf16.
@@ -513,7 +328,8 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
        !encode_2d_u8(&mx64, hidden_q, static_cast<uint64_t>(T), static_cast<uint64_t>(H), kslice, tkg::BLOCK_M / 2)) ||
       !encode_2d_u8(&mw, gate_q, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kslice, tkg::B_BOX_N))
     return TK_ERR_CUDA;
-  return launch_planned<true>(pl, dev, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, stream);
+  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns};
+  return tkg::launch_planned<true>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, stream);
 }
 
 }  // namespace
