@@ -163,3 +163,18 @@ def test_fp8_entry_point_rejects_before_cuda():
     assert f(16, 0, 16, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_INVALID_ARG         # null scale
     assert f(16, 20, 16, 16, 8, 64, 16, 2, 16, 16) == tk.TK_ERR_ALIGNMENT          # scale not 16-byte aligned
     assert f(0, 0, 0, 0, 0, 64, 16, 2, 0, 0) == tk.TK_OK                             # T == 0
+
+
+def _header_struct_fields(name):
+    import re
+    text = open(tk.exported_symbols.__globals__["HEADER"]).read()
+    body = dict((n, b) for b, n in re.findall(r"typedef struct \{([^}]*)\}\s*(\w+);", text))[name]
+    return [(t, n) for t, n in re.findall(r"^\s*(int32_t|int64_t)\s+(\w+);", body, re.M)]
+
+
+@pytest.mark.parametrize("name,binding", [("tk_gating_plan", "_Plan"), ("tk_route_plan", "_RoutePlan")])
+def test_binding_structs_match_the_header(name, binding):
+    from moe_router_gating_b200 import _binding
+    fields = getattr(_binding, binding)._fields_
+    ctype = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64}
+    assert [(n, ctype[t]) for t, n in _header_struct_fields(name)] == [(n, t) for n, t in fields]
