@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -17,7 +18,8 @@ namespace {
 
 __device__ uint32_t g_tk_error_word = 0;
 
-uint64_t g_timeout_ns = 1000000000ull;  // bounded-wait limit for kernels launched from here
+// bounded-wait limit for kernels launched from here (any host thread may set it)
+std::atomic<uint64_t> g_timeout_ns{1000000000ull};
 
 constexpr int kMaxDynamicSmem = tkg::kMaxDynamicSmem;
 constexpr int kSmemReserve = 1024 + 256;  // 1 KB alignment pad + barriers and flags
@@ -291,7 +293,7 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
                                                 tkg::BLOCK_K, tkg::BLOCK_M / 2)) ||
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
-  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns};
+  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed)};
   return tkg::launch_planned<false>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, stream);
 }
 
@@ -328,7 +330,7 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
        !encode_2d_u8(&mx64, hidden_q, static_cast<uint64_t>(T), static_cast<uint64_t>(H), kslice, tkg::BLOCK_M / 2)) ||
       !encode_2d_u8(&mw, gate_q, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kslice, tkg::B_BOX_N))
     return TK_ERR_CUDA;
-  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns};
+  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed)};
   return tkg::launch_planned<true>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, stream);
 }
 
@@ -391,7 +393,7 @@ tk_status tk_gating_device_error(uint32_t* word, int32_t clear) {
 
 tk_status tk_gating_set_wait_timeout_ns(uint64_t timeout_ns) {
   if (timeout_ns < 1000) return TK_ERR_INVALID_ARG;
-  g_timeout_ns = timeout_ns;
+  g_timeout_ns.store(timeout_ns, std::memory_order_relaxed);
   return TK_OK;
 }
 
