@@ -62,7 +62,11 @@ def launches(csv_path: str) -> str:
             continue
         v = float(r[vi].replace(",", ""))
         unit = r[ui]
-        us = v / 1000.0 if unit == "ns" else v if unit == "us" else v * 1000.0 if unit == "ms" else v
+        scale_us = {"ns": 1e-3, "nsecond": 1e-3, "us": 1.0, "usecond": 1.0, "ms": 1e3, "msecond": 1e3,
+                    "s": 1e6, "second": 1e6}
+        if unit not in scale_us:
+            raise ValueError(f"unknown time unit {unit!r} in {csv_path}")
+        us = v * scale_us[unit]
         name = r[ki].split("(")[0].strip()
         n, t = per.get(name, (0, 0.0))
         per[name] = (n + 1, t + us)
