@@ -45,7 +45,8 @@ def check_fp8(wl, duplicate_pairs=(), rows=None):
 @pytest.mark.parametrize("T,H,E,k", [
     (64, 512, 16, 2), (1, 7168, 256, 8), (128, 7168, 256, 8), (4096, 7168, 256, 8), (300, 528, 40, 3),
     (20000, 512, 256, 8), (19999, 512, 200, 8), (16384, 4096, 64, 6), (30000, 256, 512, 32), (1000, 1024, 512, 16),
-    (3, 2048, 64, 4), (129, 144, 24, 5), (200, 512, 1024, 8), (20000, 256, 768, 8),
+    (3, 2048, 64, 4), (129, 144, 24, 5), (200, 512, 1024, 8), (20000, 256, 768, 8), (300, 256, 1024, 32),
+    (24000, 128, 1016, 32),
 ])
 def test_fp8_shapes(T, H, E, k):
     check_fp8(workloads.RouterWorkload(f"fp8_{T}_{H}_{E}_{k}", T, H, E, k, seed=7))

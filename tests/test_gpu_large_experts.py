@@ -33,6 +33,7 @@ def clean_error_word():
     (20000, 512, 512, 8), (30000, 512, 320, 32), (19999, 256, 448, 5), (40000, 128, 264, 3),
     # two expert groups of up to 512 (E up to 1024), split-H and pairs
     (1, 7168, 1024, 8), (100, 1024, 640, 32), (4096, 512, 1024, 8), (20000, 256, 1024, 8), (30000, 256, 776, 16),
+    (300, 256, 1024, 32), (24000, 128, 1016, 32),
     # k up to 32 with one chunk
     (2000, 1024, 256, 32), (40000, 512, 256, 32), (5000, 256, 64, 32), (700, 256, 32, 32),
 ])
