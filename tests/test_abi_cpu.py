@@ -2,6 +2,7 @@
 host logic (validation, planning, status strings) behaves as the header says.
 No kernel is launched here."""
 import ctypes
+import os
 import subprocess
 
 import pytest
@@ -178,3 +179,31 @@ def test_binding_structs_match_the_header(name, binding):
     fields = getattr(_binding, binding)._fields_
     ctype = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64}
     assert [(n, ctype[t]) for t, n in _header_struct_fields(name)] == [(n, t) for n, t in fields]
+
+
+def test_header_is_plain_c(tmp_path):
+    # the C ABI must be usable from C: the header compiles as C99 on its own
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "tk_gating.h"\n'
+                   'int main(void) { tk_gating_plan p; tk_route_plan q; (void)p; (void)q;\n'
+                   '  return (int)sizeof(tk_status) + TK_GATING_MAX_EXPERTS + TK_ROUTE_STATIC_SCRATCH_BYTES; }\n')
+    include = os.path.dirname(tk.exported_symbols.__globals__["HEADER"])
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-fsyntax-only", "-I", include, str(src)],
+                   check=True)
+
+
+@pytest.mark.parametrize("C", [2, 4, 8, 16])
+@pytest.mark.parametrize("valid_rows", [1, 3, 31, 64, 100, 127, 128])
+def test_split_h_staging_slots_are_distinct(C, valid_rows):
+    # the exchange writes row t's partial from CTA r into owner t % C, slot (t / C) * C + r;
+    # an owner reads its n_own rows at slots [s * C, s * C + C): every write lands once, in range
+    n_own = {o: (valid_rows - o + C - 1) // C if valid_rows > o else 0 for o in range(C)}
+    seen = set()
+    for t in range(valid_rows):
+        owner = t % C
+        for r in range(C):
+            slot = (t // C) * C + r
+            assert 0 <= slot < n_own[owner] * C
+            assert (owner, slot) not in seen
+            seen.add((owner, slot))
+    assert len(seen) == sum(n * C for n in n_own.values())
