@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workload-summary", action="store_true",
+                    help="skip the per-workload table (every router workload, GPU and oracle, one GPU only)")
     ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (profiling cases)")
     ap.add_argument("--precision", default="bf16", choices=("bf16", "fp8"),
                     help="bf16 (default) or FP8 E4M3 inputs with per-token / per-expert scales")
@@ -146,7 +148,7 @@ def run_reference(args, wl):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    def __init__(self, local_rank: int, period_s: float = 0.01):
+    def __init__(self, local_rank: int, period_s: float = 0.001):
         self.samples = []
         self.period = period_s
         self._stop = threading.Event()
@@ -213,7 +215,8 @@ class ClockSampler:
             "reasons": sorted(reasons),
             "samples": len(self.samples),
             "power_w_max": max([s[3] for s in self.samples]) if self.samples else None,
-            "source": "NVML (same counters as nvidia-smi), sampled every 10 ms during the timed region",
+            "source": "NVML (same counters as nvidia-smi), sampled every %.0f ms during the timed region"
+                      % (self.period * 1e3),
         }
 
 
@@ -319,6 +322,7 @@ def run_ours(args, wl):
     sampler = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize(dev)
+    tk.clock_counters(clear=True)
     with sampler:
         if big:
             # inputs larger than L2: back-to-back launches between two events
@@ -344,6 +348,7 @@ def run_ours(args, wl):
             elapsed_ms = sum(per)
             launch_ms = elapsed_ms / args.steps
     torch.cuda.synchronize(dev)
+    kernel_clock = tk.clock_counters(clear=True)  # SM clock of the timed launches themselves
     barrier()
     err = tk.device_error(clear=True)
     if err:
@@ -391,39 +396,11 @@ def run_ours(args, wl):
 
     # ---- roofline of the (only) kernel ----
     peaks, peak_src = load_peaks()
-    bytes_alg = wl.algorithmic_bytes()
-    flops = wl.flops()
-    tc_factor = 1.0
-    if fp8:  # 1-byte operands plus the scales; the FP8 tensor peak is twice the bf16 one (nominal ratio)
-        bytes_alg = wl.T * wl.H + wl.E * wl.H + 4 * (wl.T + wl.E) + 8 * wl.T * wl.k
-        tc_factor = 2.0
-    t_s = launch_ms / 1e3
-    hbm_ach = bytes_alg / t_s / 1e9
-    tc_ach = flops / t_s / 1e12
-    # a long run of back-to-back launches settles at the power-capped clock: the
-    # tensor term then uses the sustained bf16 figure, a short one the burst figure
-    sustained = elapsed_max_ms > 100.0 and "bf16_tflops_sustained" in peaks
-    tc_peak = tc_factor * (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
-    t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (tc_peak * 1e12)
+    roofline = roofline_of(wl, launch_ms, fp8, peaks, peak_src)
     digest = kernel_source_digest()
     traffic, traffic_src = profiled_traffic(wl, digest, "_fp8" if fp8 else "")
-    hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-           "frac": hbm_ach / peaks["hbm_gbs"], "traffic": traffic}
-    tc = {"bound": "tensor", "achieved": tc_ach, "peak": tc_peak, "unit": "TFLOP/s",
-          "frac": tc_ach / tc_peak, "traffic": traffic}
-    primary, secondary = (hbm, tc) if t_hbm >= t_tc else (tc, hbm)
-    roofline = dict(primary)
-    roofline.update({
-        "peak_source": (f"{peak_src}; HBM = copy GB/s (of measured); tensor = cuBLAS bf16 "
-                        f"{'sustained (timed region > 100 ms)' if sustained else 'burst'} TFLOP/s (of measured)"
-                        + ("; x2 for FP8 (nominal FP8/bf16 ratio)" if fp8 else "")),
-        "roofline_frac": max(t_hbm, t_tc) / t_s,
-        "algorithmic_bytes_per_launch": bytes_alg, "flops_per_launch": flops,
-        "launch_ms": launch_ms, "traffic_source": traffic_src,
-        "kernel_source_digest": digest,
-        "secondary": {k: secondary[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
-    })
+    roofline["traffic"] = traffic
+    roofline.update({"traffic_source": traffic_src, "kernel_source_digest": digest})
 
     plan = tk.make_plan(wl.T, wl.H // 2 if fp8 else wl.H, wl.E, wl.k,
                         torch.cuda.get_device_properties(dev).multi_processor_count)
@@ -433,6 +410,11 @@ def run_ours(args, wl):
         v, rows, dt, cores = time_oracle(wl, args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"first {rows} of {wl.T} tokens ({dt:.1f} s, fp64 oracle with full sort, all host threads)"}
+
+    per_workload = None
+    if world == 1 and not fp8 and not args.no_workload_summary and args.tokens is None:
+        per_workload = per_workload_summary(dev, peaks, peak_src, min(args.cpu_seconds, 2.0),
+                                            not args.no_cpu_baseline)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -459,10 +441,154 @@ def run_ours(args, wl):
                          if fp8 else
                          "tk_gating_fused_topk_host: pinned host hidden -> device, kernel, scores+ids -> pinned host")},
         "gpu_launches": args.steps,
-        "clocks": sampler.summary(),
+        "clocks": clocks_summary(sampler, kernel_clock, launch_ms),
     }
+    if per_workload is not None:
+        line["workloads"] = per_workload
     print(json.dumps(line), flush=True)
     return 0
+
+
+def roofline_of(wl, launch_ms: float, fp8: bool, peaks: dict, peak_src: str) -> dict:
+    """Roofline of one launch: the binding term at the burst peaks, and the
+    fraction of the roofline at both the burst and the sustained tensor peak
+    (neither is picked by the length of the run)."""
+    bytes_alg = wl.algorithmic_bytes()
+    flops = wl.flops()
+    tc_factor = 1.0
+    if fp8:  # 1-byte operands plus the scales; the FP8 tensor peak is twice the bf16 one (nominal ratio)
+        bytes_alg = wl.T * wl.H + wl.E * wl.H + 4 * (wl.T + wl.E) + 8 * wl.T * wl.k
+        tc_factor = 2.0
+    t_s = launch_ms / 1e3
+    hbm_ach = bytes_alg / t_s / 1e9
+    tc_ach = flops / t_s / 1e12
+    tc_burst = tc_factor * peaks["bf16_tflops"]
+    tc_sust = tc_factor * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    t_hbm = bytes_alg / (peaks["hbm_gbs"] * 1e9)
+    t_tc_burst = flops / (tc_burst * 1e12)
+    t_tc_sust = flops / (tc_sust * 1e12)
+    hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+           "frac": hbm_ach / peaks["hbm_gbs"]}
+    tc = {"bound": "tensor", "achieved": tc_ach, "peak": tc_burst, "unit": "TFLOP/s", "frac": tc_ach / tc_burst}
+    primary, secondary = (hbm, tc) if t_hbm >= t_tc_burst else (tc, hbm)
+    roof = dict(primary)
+    roof.update({
+        "peak_source": (f"{peak_src}; HBM = copy GB/s (of measured); tensor = cuBLAS bf16 burst TFLOP/s "
+                        f"(of measured){'; x2 for FP8 (nominal FP8/bf16 ratio)' if fp8 else ''}"),
+        "roofline_frac": max(t_hbm, t_tc_burst) / t_s,
+        "roofline_frac_sustained": max(t_hbm, t_tc_sust) / t_s,
+        "tensor_frac_sustained": tc_ach / tc_sust,
+        "roofline_us": {"hbm": t_hbm * 1e6, "tensor_burst": t_tc_burst * 1e6, "tensor_sustained": t_tc_sust * 1e6},
+        "algorithmic_bytes_per_launch": bytes_alg, "flops_per_launch": flops, "launch_ms": launch_ms,
+        "secondary": {k: secondary[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
+    })
+    return roof
+
+
+def clocks_summary(sampler, kernel_clock: dict, launch_ms: float) -> dict:
+    """NVML samples of the timed region, plus the SM clock the launches measured
+    on themselves (first CTA: clock64 cycles over globaltimer ns)."""
+    c = sampler.summary()
+    ghz = kernel_clock.get("sm_ghz")
+    c["sm_mhz_in_kernel"] = ghz * 1e3 if ghz else None
+    c["in_kernel_launches"] = kernel_clock.get("launches")
+    c["cycles_per_launch"] = ghz * 1e9 * launch_ms / 1e3 if ghz else None
+    c["in_kernel_source"] = ("first CTA of every timed launch: SM clock64 cycles / globaltimer ns, "
+                             "summed over the launches (tk_gating_clock_counters)")
+    return c
+
+
+# The synthetic router workloads the gating is specified on, each measured in
+# the same run as the headline (one GPU): tokens/s, us per call and the roofline
+# fraction, next to the CPU oracle on a bounded sample of the same workload.
+SUMMARY_WORKLOADS = ("tiny", "deepseek", "skew", "train", "decode_T1", "decode_T8", "decode_T32", "decode_T128",
+                     "decode_T256")
+
+
+def time_calls(step, stream, steps: int, flush) -> float:
+    """Mean ms per call: each call timed alone with CUDA events after an L2 flush
+    (flush is None for inputs larger than L2: back-to-back calls between two events)."""
+    import torch
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if flush is None:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / steps
+
+
+def oracle_single_thread_rate(wl, seconds: float):
+    """The oracle's tokens/s with one OpenMP thread (the same code, one core)."""
+    import ctypes
+    gomp = ctypes.CDLL("libgomp.so.1")
+    before = gomp.omp_get_max_threads()
+    gomp.omp_set_num_threads(1)
+    try:
+        v, rows, dt, _ = time_oracle(wl, seconds)
+    finally:
+        gomp.omp_set_num_threads(before)
+    return v, rows, dt
+
+
+def per_workload_summary(dev, peaks, peak_src, cpu_seconds: float, with_cpu: bool) -> dict:
+    import torch
+
+    import moe_router_gating_b200 as tk
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    for name in SUMMARY_WORKLOADS:
+        wl = workloads.WORKLOADS[name]
+        x = workloads.to_torch_bf16(wl.hidden()).to(dev)
+        w = workloads.to_torch_bf16(wl.gate_weight()).to(dev)
+        s = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+        i = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+        big = wl.T * wl.H * 2 > L2_BYTES
+
+        def step():
+            tk.fused_topk_gating(x, w, wl.k, scores=s, ids=i, stream=stream)
+        tk.clock_counters(clear=True)
+        steps = 20 if big else 200
+        ms = time_calls(step, stream, steps, None if big else flush)
+        clk = tk.clock_counters(clear=True)
+        roof = roofline_of(wl, ms, False, peaks, peak_src)
+        entry = {"T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "us_per_call": ms * 1e3,
+                 "tokens_per_s": wl.T / (ms / 1e3),
+                 "timing": ("back-to-back calls, inputs larger than L2" if big else
+                            "each call alone after an L2 flush (256 MB write), mean of %d" % steps),
+                 "roofline": {"bound": roof["bound"], "frac": roof["frac"], "roofline_frac": roof["roofline_frac"],
+                              "roofline_frac_sustained": roof["roofline_frac_sustained"],
+                              "roofline_us": roof["roofline_us"]},
+                 "sm_mhz_in_kernel": clk["sm_ghz"] * 1e3 if clk["sm_ghz"] else None,
+                 "plan": {k: v for k, v in tk.make_plan(wl.T, wl.H, wl.E, wl.k,
+                                                        torch.cuda.get_device_properties(dev).multi_processor_count)
+                          .items() if k in ("variant", "cluster", "grid", "num_tiles", "num_half_tiles")}}
+        if err := tk.device_error(clear=True):
+            raise SystemExit(f"device error word {err:#x} during the {name} summary")
+        if with_cpu:
+            v, rows, dt, cores = time_oracle(wl, cpu_seconds)
+            entry["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                     "sample": f"first {rows} of {wl.T} tokens ({dt:.2f} s)"}
+            if name == "deepseek":
+                v1, rows1, dt1 = oracle_single_thread_rate(wl, cpu_seconds)
+                entry["cpu_baseline_1thread"] = {"value": v1, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                                 "sample": f"first {rows1} of {wl.T} tokens ({dt1:.2f} s)"}
+        out[name] = entry
+        del x, w, s, i
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -141,6 +141,31 @@ TK_API tk_status tk_gating_fused_topk_fp8(const void* hidden_q, const float* hid
                                           const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k,
                                           float* scores, int32_t* ids, void* stream);
 
+/*
+ * tk_gating_fused_topk_logits / tk_gating_fused_topk_fp8_logits -- the same
+ * operators, which also store every logit their selection ranked.
+ *
+ * A verification aid for the logits step of section 4.1 (logits =
+ * hidden_states @ gate_weight, here in fp32 on the tensor cores): the launch
+ * is the one tk_gating_fused_topk (or _fp8) makes, the same kernels, whose
+ * epilogue additionally writes each fp32 logit it offers to the selection
+ * (FP8: after both scales).  scores and ids are bitwise the ones the plain
+ * call returns.  Not for production use: it writes T x E x 4 bytes more.
+ *
+ *   logits   device, out fp32 [T, E] row-major, 16-byte aligned.
+ *   the other arguments as tk_gating_fused_topk (or _fp8).
+ *
+ * Errors as tk_gating_fused_topk (or _fp8); TK_ERR_INVALID_ARG for a null
+ * logits when T > 0, TK_ERR_ALIGNMENT when it is not 16-byte aligned.
+ */
+TK_API tk_status tk_gating_fused_topk_logits(const void* hidden, const void* gate_weight, int64_t T, int64_t H,
+                                             int64_t E, int32_t k, float* scores, int32_t* ids, float* logits,
+                                             void* stream);
+TK_API tk_status tk_gating_fused_topk_fp8_logits(const void* hidden_q, const float* hidden_scale,
+                                                 const void* gate_q, const float* gate_scale, int64_t T, int64_t H,
+                                                 int64_t E, int32_t k, float* scores, int32_t* ids, float* logits,
+                                                 void* stream);
+
 /* Kernel variants chosen by the planner. */
 typedef enum {
   TK_VARIANT_NONE = 0,        /* T == 0: nothing to launch */
@@ -186,6 +211,20 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
  * TK_ERR_DEVICE_TIMEOUT when the word is non-zero, TK_OK otherwise.
  */
 TK_API tk_status tk_gating_device_error(uint32_t* word, int32_t clear);
+
+/*
+ * tk_gating_clock_counters -- SM-clock record of the fused gating launches on
+ * the current device.  The first CTA of every launch of tk_gating_fused_topk
+ * (and of its variants) adds the SM clock cycles and the nanoseconds from its
+ * start to its end, and 1, to three device counters; this call reads them into
+ * *sm_cycles, *elapsed_ns and *launches, and zeroes them when `clear` is
+ * non-zero.  sm_cycles / elapsed_ns is the mean SM clock (GHz) under the
+ * launches' own load -- a measurement aid for timing.  Synchronises the
+ * device.  TK_ERR_INVALID_ARG for a null pointer, TK_ERR_CUDA when a CUDA call
+ * fails.  Counters of a device no gating call has run on read as zero.
+ */
+TK_API tk_status tk_gating_clock_counters(uint64_t* sm_cycles, uint64_t* elapsed_ns, uint64_t* launches,
+                                          int32_t clear);
 
 /*
  * tk_gating_set_wait_timeout_ns -- limit (nanoseconds) of every bounded wait in

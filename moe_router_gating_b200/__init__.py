@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     TK_ERR_INVALID_ARG,
     TK_ERR_UNSUPPORTED,
     TkGatingError,
+    clock_counters,
     device_error,
     exported_symbols,
     fused_topk_gating,
@@ -40,6 +41,6 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "fused_topk_gating", "fused_topk_gating_fp8", "fused_topk_gating_host", "fused_topk_gating_ptr", "make_plan", "route", "route_plan",
-    "route_ptr", "device_error",
+    "route_ptr", "route_static_ptr", "device_error", "clock_counters",
     "set_wait_timeout_ns", "status_string", "TkGatingError", "library", "library_path",
 ]

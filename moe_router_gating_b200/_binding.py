@@ -60,6 +60,13 @@ def library() -> ctypes.CDLL:
             lib.tk_gating_fused_topk_host.restype = ctypes.c_int
             lib.tk_gating_fused_topk_fp8.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp]
             lib.tk_gating_fused_topk_fp8.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_logits.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
+            lib.tk_gating_fused_topk_logits.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_fp8_logits.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
+            lib.tk_gating_fused_topk_fp8_logits.restype = ctypes.c_int
+            u64p = ctypes.POINTER(ctypes.c_uint64)
+            lib.tk_gating_clock_counters.argtypes = [u64p, u64p, u64p, i32]
+            lib.tk_gating_clock_counters.restype = ctypes.c_int
             lib.tk_gating_make_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(_Plan)]
             lib.tk_gating_make_plan.restype = ctypes.c_int
             lib.tk_gating_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -106,12 +113,14 @@ def fused_topk_gating_ptr(hidden: int, gate_weight: int, T: int, H: int, E: int,
     return int(library().tk_gating_fused_topk(hidden, gate_weight, T, H, E, k, scores, ids, stream))
 
 
-def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, stream=None):
+def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, stream=None, logits=None):
     """``(scores[T,k] fp32, ids[T,k] int32) = softmax(topk(hidden @ gate_weight))``.
 
     ``hidden`` is a CUDA bf16 ``[T, H]`` tensor and ``gate_weight`` a CUDA bf16
     ``[H, E]`` tensor, both contiguous.  Output tensors may be passed in.  The
-    launch goes on ``stream`` (default: the current torch stream).
+    launch goes on ``stream`` (default: the current torch stream).  Passing a
+    contiguous fp32 ``[T, E]`` CUDA tensor as ``logits`` calls the verification
+    entry point, which also stores every logit the selection ranked.
     """
     import torch
     if hidden.dtype != torch.bfloat16 or gate_weight.dtype != torch.bfloat16:
@@ -133,13 +142,25 @@ def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, st
         raise ValueError("scores must be fp32 [T,k] and ids int32 [T,k], contiguous")
     lib = library()
     args = (hidden.data_ptr(), gate_weight.data_ptr(), T, H, E, int(top_k), scores.data_ptr(), ids.data_ptr())
+    fn, name = lib.tk_gating_fused_topk, "tk_gating_fused_topk"
+    if logits is not None:
+        _check_logits(logits, T, E, hidden.device)
+        args = args + (logits.data_ptr(),)
+        fn, name = lib.tk_gating_fused_topk_logits, "tk_gating_fused_topk_logits"
     if hidden.device.index == torch.cuda.current_device():
-        st = lib.tk_gating_fused_topk(*args, _stream_handle(stream, hidden.device))
+        st = fn(*args, _stream_handle(stream, hidden.device))
     else:
         with torch.cuda.device(hidden.device):
-            st = lib.tk_gating_fused_topk(*args, _stream_handle(stream, hidden.device))
-    _check(st, "tk_gating_fused_topk")
+            st = fn(*args, _stream_handle(stream, hidden.device))
+    _check(st, name)
     return scores, ids
+
+
+def _check_logits(logits, T: int, E: int, device) -> None:
+    import torch
+    if logits.dtype != torch.float32 or tuple(logits.shape) != (T, E) or not logits.is_contiguous() \
+            or logits.device != device:
+        raise ValueError(f"logits must be a contiguous fp32 [{T}, {E}] tensor on {device}")
 
 
 def fused_topk_gating_fp8_ptr(hidden_q: int, hidden_scale: int, gate_q: int, gate_scale: int, T: int, H: int,
@@ -150,10 +171,12 @@ def fused_topk_gating_fp8_ptr(hidden_q: int, hidden_scale: int, gate_q: int, gat
 
 
 def fused_topk_gating_fp8(hidden_q, hidden_scale, gate_q, gate_scale, top_k: int, scores=None, ids=None,
-                          stream=None):
+                          stream=None, logits=None):
     """Fused gating on FP8 E4M3 inputs: ``hidden_q`` [T, H] and ``gate_q`` [E, H]
     (expert-major) as torch.float8_e4m3fn or torch.uint8 CUDA tensors, with fp32
-    ``hidden_scale`` [T] and ``gate_scale`` [E].  Returns ``(scores, ids)``."""
+    ``hidden_scale`` [T] and ``gate_scale`` [E].  Returns ``(scores, ids)``.
+    ``logits`` (fp32 [T, E]) selects the verification entry point, which also
+    stores every scaled logit the selection ranked."""
     import torch
     fp8_types = (torch.float8_e4m3fn, torch.uint8)
     if hidden_q.dtype not in fp8_types or gate_q.dtype not in fp8_types:
@@ -173,11 +196,16 @@ def fused_topk_gating_fp8(hidden_q, hidden_scale, gate_q, gate_scale, top_k: int
         scores = torch.empty((T, top_k), dtype=torch.float32, device=hidden_q.device)
     if ids is None:
         ids = torch.empty((T, top_k), dtype=torch.int32, device=hidden_q.device)
+    args = (hidden_q.data_ptr(), hidden_scale.data_ptr(), gate_q.data_ptr(), gate_scale.data_ptr(), T, H, E,
+            int(top_k), scores.data_ptr(), ids.data_ptr())
+    fn, name = library().tk_gating_fused_topk_fp8, "tk_gating_fused_topk_fp8"
+    if logits is not None:
+        _check_logits(logits, T, E, hidden_q.device)
+        args = args + (logits.data_ptr(),)
+        fn, name = library().tk_gating_fused_topk_fp8_logits, "tk_gating_fused_topk_fp8_logits"
     with torch.cuda.device(hidden_q.device):
-        st = library().tk_gating_fused_topk_fp8(
-            hidden_q.data_ptr(), hidden_scale.data_ptr(), gate_q.data_ptr(), gate_scale.data_ptr(), T, H, E,
-            int(top_k), scores.data_ptr(), ids.data_ptr(), _stream_handle(stream, hidden_q.device))
-    _check(st, "tk_gating_fused_topk_fp8")
+        st = fn(*args, _stream_handle(stream, hidden_q.device))
+    _check(st, name)
     return scores, ids
 
 
@@ -211,6 +239,17 @@ def device_error(clear: bool = True) -> int:
     if st not in (TK_OK, TK_ERR_DEVICE_TIMEOUT):
         _check(st, "tk_gating_device_error")
     return int(w.value)
+
+
+def clock_counters(clear: bool = True) -> dict:
+    """SM-clock record of the gating launches on the current device since the
+    last clear: ``{"sm_cycles", "elapsed_ns", "launches", "sm_ghz"}`` (first CTA
+    of each launch, start to end; ``sm_ghz`` = cycles / ns, None without launches)."""
+    c, n, l = ctypes.c_uint64(0), ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check(library().tk_gating_clock_counters(ctypes.byref(c), ctypes.byref(n), ctypes.byref(l), 1 if clear else 0),
+           "tk_gating_clock_counters")
+    return {"sm_cycles": int(c.value), "elapsed_ns": int(n.value), "launches": int(l.value),
+            "sm_ghz": (c.value / n.value) if n.value else None}
 
 
 def set_wait_timeout_ns(timeout_ns: int) -> None:

@@ -7,7 +7,7 @@ namespace tkg {
 template bool set_up_gating_kernels<false>();
 template tk_status launch_planned<false>(const tk_gating_plan&, const LaunchEnv&, const CUtensorMap&,
                                          const CUtensorMap&, const CUtensorMap&, int64_t, int64_t, int64_t, int32_t,
-                                         float*, int32_t*, const float*, const float*, cudaStream_t);
+                                         float*, int32_t*, const float*, const float*, float*, cudaStream_t);
 
 void measure_split_cluster_capacity(int counts[4]) {
   for (int i = 1; i <= 4; ++i) {

@@ -27,6 +27,7 @@ struct LaunchEnv {
   int max_split_cluster;  // largest split-H cluster the device co-schedules
   uint32_t* err_word;     // device error word of the bounded waits
   uint64_t timeout_ns;    // bounded-wait limit
+  uint64_t* clock;        // SM-clock counters of the launches (cycles, ns, launches)
 };
 
 // Shared-memory limits (and non-portable cluster sizes) of every kernel instance
@@ -35,20 +36,24 @@ template <bool FP8>
 bool set_up_gating_kernels();
 
 // Launch the planned kernel on encoded maps.  FP8: hscale / gscale are the
-// per-token and per-expert scales (unused for bf16).
+// per-token and per-expert scales (unused for bf16).  logits: optional fp32
+// [T, E] that also receives every logit the selection ranks (verification).
 template <bool FP8>
 tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const CUtensorMap& mx,
                          const CUtensorMap& mx64, const CUtensorMap& mw, int64_t T, int64_t H, int64_t E, int32_t k,
-                         float* scores, int32_t* ids, const float* hscale, const float* gscale, cudaStream_t stream);
+                         float* scores, int32_t* ids, const float* hscale, const float* gscale, float* logits,
+                         cudaStream_t stream);
 
 extern template bool set_up_gating_kernels<false>();
 extern template bool set_up_gating_kernels<true>();
 extern template tk_status launch_planned<false>(const tk_gating_plan&, const LaunchEnv&, const CUtensorMap&,
                                                 const CUtensorMap&, const CUtensorMap&, int64_t, int64_t, int64_t,
-                                                int32_t, float*, int32_t*, const float*, const float*, cudaStream_t);
+                                                int32_t, float*, int32_t*, const float*, const float*, float*,
+                                                cudaStream_t);
 extern template tk_status launch_planned<true>(const tk_gating_plan&, const LaunchEnv&, const CUtensorMap&,
                                                const CUtensorMap&, const CUtensorMap&, int64_t, int64_t, int64_t,
-                                               int32_t, float*, int32_t*, const float*, const float*, cudaStream_t);
+                                               int32_t, float*, int32_t*, const float*, const float*, float*,
+                                               cudaStream_t);
 
 // Clusters of 2, 4, 8 and 16 full-shared-memory split-H CTAs that the current
 // device runs at once, into counts[0..3] (0 where a size cannot run).

@@ -101,7 +101,8 @@ tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, co
 template <bool FP8>
 tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const CUtensorMap& mx,
                          const CUtensorMap& mx64, const CUtensorMap& mw, int64_t T, int64_t H, int64_t E, int32_t k,
-                         float* scores, int32_t* ids, const float* hscale, const float* gscale, cudaStream_t stream) {
+                         float* scores, int32_t* ids, const float* hscale, const float* gscale, float* logits,
+                         cudaStream_t stream) {
   uint32_t* err = env.err_word;
   if (pl.variant == TK_VARIANT_SPLIT_H) {
     SplitHParams sp;
@@ -124,6 +125,8 @@ tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const C
     sp.err_word = err;
     sp.hscale = hscale;
     sp.gscale = gscale;
+    sp.logits = logits;
+    sp.clock = env.clock;
     const int mc = env.max_split_cluster;
     // lists of 4 also serve k = 1, 2 (fewer kernel instances to build; an
     // insertion into 4 slots costs little more than into 1 or 2)
@@ -155,6 +158,8 @@ tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const C
   prm.err_word = err;
   prm.hscale = hscale;
   prm.gscale = gscale;
+  prm.logits = logits;
+  prm.clock = env.clock;
 
   if (k <= 4) return launch_row_variant<4, FP8>(pl, mx, mx64, mw, prm, stream);
   if (k <= 8) return launch_row_variant<8, FP8>(pl, mx, mx64, mw, prm, stream);

@@ -91,6 +91,8 @@ struct RowTileParams {
   uint32_t* err_word;
   const float* hscale;  // FP8 only: per-token scales [T]
   const float* gscale;  // FP8 only: per-expert scales [E]
+  float* logits;        // optional [T, E]: every logit the selection ranks is also stored (verification)
+  uint64_t* clock;      // SM-clock counters: the first CTA adds its cycles and ns (and 1) per launch
 };
 
 // K elements of H per K slice: one 128-byte swizzle row of bf16 or of FP8 values.
@@ -218,6 +220,16 @@ __device__ __forceinline__ bool tile_work(const RowTileParams& p, int unit, int 
 // Offer 32 consecutive logits (accumulator columns c0 .. c0+31, expert ids
 // col_base + c0 ..) of this thread's row; columns at or beyond ncols (MMA
 // padding) are skipped.
+// Verification aid: store 32 consecutive logits of one row (experts e0 ..
+// e0+31, those below `limit`) into the row-major [T, E] array `logits`.
+__device__ __forceinline__ void store_logit_chunk(float* logits, int64_t row, int E, int e0, int limit,
+                                                  const uint32_t (&r)[32]) {
+  float* dst = logits + row * E + e0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (e0 + j < limit) dst[j] = __uint_as_float(r[j]);
+}
+
 template <int KMAX>
 __device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (&r)[32], int c0, int ncols,
                                             int col_base) {
@@ -240,6 +252,9 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
                             const __grid_constant__ CUtensorMap map_w, const RowTileParams p) {
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
   constexpr bool kPair = CG == 2;
+  const bool clock_cta = p.clock != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
+  const uint64_t t0_ns = clock_cta ? globaltimer_ns() : 0;
+  const uint64_t t0_clk = clock_cta ? sm_clock64() : 0;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align_1024(smem_dyn);
   uint8_t* sA = smem;
@@ -459,8 +474,11 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     for (; tile_work<CG, EG>(p, unit, units, local, w); ++local) {
       const uint32_t buf = static_cast<uint32_t>(local % p.acc_bufs);
       const uint32_t acc_phase = static_cast<uint32_t>(local / p.acc_bufs) & 1;
-      bool ok = mbar_wait(&acc_full[buf], acc_phase, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      const bool ok = mbar_wait(&acc_full[buf], acc_phase, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
+      // The four epilogue warps take one decision: a warp that went on alone
+      // after the others gave up would wait for them forever at the half
+      // tile's list exchange below.
+      if (!named_barrier_and(2, NUM_EPI_WARPS * 32, ok)) break;
       tc_fence_after_sync();
 
       // full tile: one row per thread, TMEM column c = expert e0 + c of the group;
@@ -471,12 +489,11 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       if (w.eg == 0) top.reset();  // the lists run over every expert group of the tile
       const uint32_t acc_addr = lane_base + buf * p.acc_stride;
       const GroupShape gs = group_shape(p, w.eg);
+      const int64_t my_row = w.half ? static_cast<int64_t>(w.row0) + rank * (BLOCK_M / 2) + (quad & 1) * 32 + lane
+                                    : static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
       float hs = 1.0f;  // FP8: this row's token scale
-      if constexpr (FP8) {
-        const int64_t my_row = w.half ? static_cast<int64_t>(w.row0) + rank * (BLOCK_M / 2) + (quad & 1) * 32 + lane
-                                      : static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
-        hs = my_row < p.T ? __ldg(p.hscale + my_row) : 0.0f;
-      }
+      if constexpr (FP8) hs = my_row < p.T ? __ldg(p.hscale + my_row) : 0.0f;
+      const bool dump = p.logits != nullptr && my_row < p.T;
       // full tiles: one pass over the group's columns; half tiles: one per chunk
       const int passes = w.half ? gs.n_chunks : 1;
       for (int c = 0; c < passes; ++c) {
@@ -495,9 +512,11 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           if (second) tmem_ld_32(chunk_addr + c0 + 32, r1);
           tmem_ld_wait();
           scale_chunk<FP8>(r0, p.gscale, col_base + c0, p.E, hs);
+          if (dump) store_logit_chunk(p.logits, my_row, p.E, col_base + c0, col_base + ncols, r0);
           offer_chunk(top, r0, c0, ncols, col_base);
           if (second) {
             scale_chunk<FP8>(r1, p.gscale, col_base + c0 + 32, p.E, hs);
+            if (dump) store_logit_chunk(p.logits, my_row, p.E, col_base + c0 + 32, col_base + ncols, r1);
             offer_chunk(top, r1, c0 + 32, ncols, col_base);
           }
         }
@@ -564,6 +583,7 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     else
       tmem_dealloc(tmem_base, p.tmem_cols);
   }
+  if (clock_cta) record_launch_clock(p.clock, t0_ns, t0_clk);
 }
 
 }  // namespace tkg

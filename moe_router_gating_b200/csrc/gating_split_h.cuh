@@ -31,7 +31,8 @@
 // expert-major gate, 128 K values per slice); owners scale the summed logits
 // by the token's and the expert's scale before selecting.
 //
-// Nothing but scores and ids is written to global memory.
+// Nothing but scores and ids is written to global memory (and, when the
+// verification array `logits` is given, every summed logit of the tile).
 #pragma once
 
 #include <cuda.h>
@@ -69,12 +70,17 @@ struct SplitHParams {
   uint32_t* err_word;
   const float* hscale;  // FP8 only: per-token scales [T]
   const float* gscale;  // FP8 only: per-expert scales [E]
+  float* logits;        // optional [T, E]: every logit the selection ranks is also stored (verification)
+  uint64_t* clock;      // SM-clock counters: the first CTA adds its cycles and ns (and 1) per launch
 };
 
 template <int KMAX, int C, bool FP8>
 __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     gating_split_h_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                           const SplitHParams p) {
+  const bool clock_cta = p.clock != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
+  const uint64_t t0_ns = clock_cta ? globaltimer_ns() : 0;
+  const uint64_t t0_clk = clock_cta ? sm_clock64() : 0;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = align_1024(smem_dyn);
   uint8_t* sA = smem;
@@ -149,7 +155,8 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
         const uint64_t pol_w = l2_policy_evict_last();
         const uint32_t slice_tx = A_STAGE_BYTES + boxes * B_BOX_BYTES;
         int issued = 0;
-        for (int kb = kb0; kb < kb1; kb += p.kps) {
+        // after an abort no later expert group is loaded
+        for (int kb = *abort_flag ? kb1 : kb0; kb < kb1; kb += p.kps) {
           // a stage holds up to kps slices, never past this CTA's H slice
           const int n_sub = min(p.kps, kb1 - kb);
           if (!mbar_wait(&empty[ring_stage], ring_phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER,
@@ -193,8 +200,9 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
         const uint32_t idesc0 = mma_idesc<FP8>(BLOCK_M, min(np, N_CHUNK));
         const uint32_t idesc1 = mma_idesc<FP8>(BLOCK_M, np > N_CHUNK ? np - N_CHUNK : N_CHUNK);
         const bool two_chunks = n_chunks > 1;
-        bool ok = true;
-        for (int kb = kb0; kb < kb1; kb += p.kps) {
+        // after an abort no later expert group is computed
+        bool ok = *abort_flag == 0;
+        for (int kb = kb0; ok && kb < kb1; kb += p.kps) {
           const int n_sub = min(p.kps, kb1 - kb);
           if (!mbar_wait(&full[ring_stage], ring_phase, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) {
             ok = false;
@@ -228,7 +236,9 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
             ring_phase ^= 1;
           }
         }
-        if (ok) umma_commit(acc_full);
+        // committed for every group, finished or not, so that the barrier's
+        // phases follow the groups; the push warps check the abort flag
+        umma_commit(acc_full);
         umma_commit(drain);
         mbar_wait(drain, parity, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
       }
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     bool acc_ok = true;
     if (push_warp) {
       acc_ok = mbar_wait(acc_full, parity, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
-      acc_ok = __all_sync(0xffffffffu, acc_ok);
+      acc_ok = __all_sync(0xffffffffu, acc_ok && *abort_flag == 0);
     }
 
     for (int pass = 0; pass < n_chunks; ++pass) {
@@ -338,8 +348,17 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
           }
           return acc;
         };
+        float* dump = p.logits == nullptr ? nullptr
+                                          : p.logits + (static_cast<int64_t>(tile) * BLOCK_M + static_cast<int>(r) +
+                                                        C * slot) * p.E + ebase;
         for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
           const float4 acc = column_quad(c);
+          if (dump != nullptr) {
+            dump[c] = acc.x;
+            if (c + 1 < pass_cols) dump[c + 1] = acc.y;
+            if (c + 2 < pass_cols) dump[c + 2] = acc.z;
+            if (c + 3 < pass_cols) dump[c + 3] = acc.w;
+          }
           top.offer(acc.x, ebase + c);
           if (c + 1 < pass_cols) top.offer(acc.y, ebase + c + 1);
           if (c + 2 < pass_cols) top.offer(acc.z, ebase + c + 2);
@@ -359,6 +378,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     const int64_t row = static_cast<int64_t>(tile) * BLOCK_M + t_local;
     top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
   }
+  if (clock_cta) record_launch_clock(p.clock, t0_ns, t0_clk);
 }
 
 }  // namespace tkg

@@ -40,6 +40,24 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+__device__ __forceinline__ uint64_t sm_clock64() {
+  uint64_t c;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+  return c;
+}
+
+// SM-clock counters of the gating launches: clock[0] += SM cycles and
+// clock[1] += nanoseconds from (t0_clk, t0_ns) to now, clock[2] += 1.  Their
+// ratio is the mean SM clock under the launches' own load.
+__device__ __forceinline__ void record_launch_clock(uint64_t* clock, uint64_t t0_ns, uint64_t t0_clk) {
+  const uint64_t clk = sm_clock64();
+  const uint64_t ns = globaltimer_ns();
+  unsigned long long* c = reinterpret_cast<unsigned long long*>(clock);
+  atomicAdd(c, static_cast<unsigned long long>(clk - t0_clk));
+  atomicAdd(c + 1, static_cast<unsigned long long>(ns - t0_ns));
+  atomicAdd(c + 2, 1ull);
+}
+
 __device__ __forceinline__ uint32_t lane_id() {
   uint32_t l;
   asm volatile("mov.u32 %0, %%laneid;" : "=r"(l));
@@ -374,6 +392,21 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t smem_addr, uint32_t
 // Named barrier among `count` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier among `count` threads that also ANDs `pred` over them: every
+// participant gets true only when every participant passed true.
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 // Arrive on an mbarrier of another CTA of the cluster (address from mapa).

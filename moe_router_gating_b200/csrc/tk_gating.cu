@@ -17,6 +17,9 @@
 namespace {
 
 __device__ uint32_t g_tk_error_word = 0;
+// SM cycles, nanoseconds and launches of the gating kernels (first CTA of each
+// launch), summed until tk_gating_clock_counters clears them.
+__device__ uint64_t g_tk_clock[3] = {0, 0, 0};
 
 // bounded-wait limit for kernels launched from here (any host thread may set it)
 std::atomic<uint64_t> g_timeout_ns{1000000000ull};
@@ -225,6 +228,7 @@ struct DeviceState {
   tk_status status = TK_OK;
   int num_sms = 0;
   uint32_t* err_word = nullptr;
+  uint64_t* clock = nullptr;
   int max_split_cluster = 0;
   ClusterCapacity capacity = {};
 };
@@ -252,12 +256,15 @@ const DeviceState* device_state() {
     return &d;
   }
   void* err = nullptr;
-  if (cudaGetSymbolAddress(&err, g_tk_error_word) != cudaSuccess || !tkg::set_up_gating_kernels<false>() ||
+  void* clk = nullptr;
+  if (cudaGetSymbolAddress(&err, g_tk_error_word) != cudaSuccess ||
+      cudaGetSymbolAddress(&clk, g_tk_clock) != cudaSuccess || !tkg::set_up_gating_kernels<false>() ||
       !tkg::set_up_gating_kernels<true>()) {
     cudaGetLastError();
     return nullptr;  // not cached: a later call retries
   }
   d.err_word = static_cast<uint32_t*>(err);
+  d.clock = static_cast<uint64_t*>(clk);
   d.capacity.n[0] = d.num_sms;
   tkg::measure_split_cluster_capacity(d.capacity.n + 1);
   d.max_split_cluster = 0;
@@ -272,7 +279,7 @@ const DeviceState* device_state() {
 }
 
 tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int64_t H, int64_t E, int32_t k,
-                            float* scores, int32_t* ids, cudaStream_t stream) {
+                            float* scores, int32_t* ids, float* logits, cudaStream_t stream) {
   tk_status st = validate_sizes(T, H, E, k);
   if (st != TK_OK) return st;
   if (T == 0) return TK_OK;
@@ -293,8 +300,9 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
                                                 tkg::BLOCK_K, tkg::BLOCK_M / 2)) ||
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
-  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed)};
-  return tkg::launch_planned<false>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, stream);
+  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
+                           dev->clock};
+  return tkg::launch_planned<false>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, logits, stream);
 }
 
 // FP8 sizes: H a multiple of 16 (16-byte rows of 8-bit values); E and k as bf16.
@@ -306,7 +314,7 @@ tk_status validate_sizes_fp8(int64_t T, int64_t H, int64_t E, int32_t k) {
 
 tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale, const void* gate_q,
                                 const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k, float* scores,
-                                int32_t* ids, cudaStream_t stream) {
+                                int32_t* ids, float* logits, cudaStream_t stream) {
   tk_status st = validate_sizes_fp8(T, H, E, k);
   if (st != TK_OK) return st;
   if (T == 0) return TK_OK;
@@ -330,8 +338,10 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
        !encode_2d_u8(&mx64, hidden_q, static_cast<uint64_t>(T), static_cast<uint64_t>(H), kslice, tkg::BLOCK_M / 2)) ||
       !encode_2d_u8(&mw, gate_q, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kslice, tkg::B_BOX_N))
     return TK_ERR_CUDA;
-  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed)};
-  return tkg::launch_planned<true>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, stream);
+  const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
+                           dev->clock};
+  return tkg::launch_planned<true>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, logits,
+                                   stream);
 }
 
 }  // namespace
@@ -340,7 +350,16 @@ extern "C" {
 
 tk_status tk_gating_fused_topk(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,
                                int32_t k, float* scores, int32_t* ids, void* stream) {
-  return fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, static_cast<cudaStream_t>(stream));
+  return fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+tk_status tk_gating_fused_topk_logits(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,
+                                      int32_t k, float* scores, int32_t* ids, float* logits, void* stream) {
+  const tk_status st = validate_sizes(T, H, E, k);
+  if (st != TK_OK || T == 0) return st;
+  if (logits == nullptr) return TK_ERR_INVALID_ARG;
+  if (!aligned16(logits)) return TK_ERR_ALIGNMENT;
+  return fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, logits, static_cast<cudaStream_t>(stream));
 }
 
 tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* gate_weight, int64_t T, int64_t H,
@@ -358,7 +377,7 @@ tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* gate_we
   const size_t out_bytes = static_cast<size_t>(T) * static_cast<size_t>(k) * 4;
   if (cudaMemcpyAsync(hidden_dev, hidden_host, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return TK_ERR_CUDA;
-  st = fused_topk_device(hidden_dev, gate_weight, T, H, E, k, scores_dev, ids_dev, s);
+  st = fused_topk_device(hidden_dev, gate_weight, T, H, E, k, scores_dev, ids_dev, nullptr, s);
   if (st != TK_OK) return st;
   if (cudaMemcpyAsync(scores_host, scores_dev, out_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
       cudaMemcpyAsync(ids_host, ids_dev, out_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -369,7 +388,18 @@ tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* gate_we
 tk_status tk_gating_fused_topk_fp8(const void* hidden_q, const float* hidden_scale, const void* gate_q,
                                    const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k, float* scores,
                                    int32_t* ids, void* stream) {
-  return fused_topk_fp8_device(hidden_q, hidden_scale, gate_q, gate_scale, T, H, E, k, scores, ids,
+  return fused_topk_fp8_device(hidden_q, hidden_scale, gate_q, gate_scale, T, H, E, k, scores, ids, nullptr,
+                               static_cast<cudaStream_t>(stream));
+}
+
+tk_status tk_gating_fused_topk_fp8_logits(const void* hidden_q, const float* hidden_scale, const void* gate_q,
+                                          const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k,
+                                          float* scores, int32_t* ids, float* logits, void* stream) {
+  const tk_status st = validate_sizes_fp8(T, H, E, k);
+  if (st != TK_OK || T == 0) return st;
+  if (logits == nullptr) return TK_ERR_INVALID_ARG;
+  if (!aligned16(logits)) return TK_ERR_ALIGNMENT;
+  return fused_topk_fp8_device(hidden_q, hidden_scale, gate_q, gate_scale, T, H, E, k, scores, ids, logits,
                                static_cast<cudaStream_t>(stream));
 }
 
@@ -389,6 +419,21 @@ tk_status tk_gating_device_error(uint32_t* word, int32_t clear) {
   }
   *word = w;
   return w ? TK_ERR_DEVICE_TIMEOUT : TK_OK;
+}
+
+tk_status tk_gating_clock_counters(uint64_t* sm_cycles, uint64_t* elapsed_ns, uint64_t* launches, int32_t clear) {
+  if (sm_cycles == nullptr || elapsed_ns == nullptr || launches == nullptr) return TK_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return TK_ERR_CUDA;
+  uint64_t c[3] = {0, 0, 0};
+  if (cudaMemcpyFromSymbol(c, g_tk_clock, sizeof(c)) != cudaSuccess) return TK_ERR_CUDA;
+  if (clear) {
+    const uint64_t zero[3] = {0, 0, 0};
+    if (cudaMemcpyToSymbol(g_tk_clock, zero, sizeof(zero)) != cudaSuccess) return TK_ERR_CUDA;
+  }
+  *sm_cycles = c[0];
+  *elapsed_ns = c[1];
+  *launches = c[2];
+  return TK_OK;
 }
 
 tk_status tk_gating_set_wait_timeout_ns(uint64_t timeout_ns) {

@@ -91,3 +91,48 @@ def check(gpu_scores: np.ndarray, gpu_ids: np.ndarray, oracle_result, rows=None,
             assert pa < pb, f"{label}: duplicate {b} ranked before {a} on row {rows[t]}"
     return {"rows": int(T), "wide_gap_rows": int(wide.sum()), "reordered_rows": swaps,
             "max_score_err": float(err)}
+
+
+# The kernels' fp32 logits against the oracle's fp64 logits.  A logit sums
+# H = 7168 exact bf16 products in H / 16 = 448 fp32 tensor-core steps (FP8:
+# 224); each step rounds a running sum of magnitude <~ 4 at relative 2^-24,
+# about 2.4e-7.  Modelled as a random walk of those roundings the error has
+# sigma ~ sqrt(448) * 2.4e-7 / 2 ~ 2.5e-6; the largest of tens of millions of
+# logits lies several sigma out.  Measured on B200 (every logit of each
+# workload): at most 5.4e-5 (65536 x 7168 x 1024), 5.0e-5 (65536 x 7168 x 256),
+# 9.4e-6 (4096 x 7168 x 256), 1.4e-6 (one token); FP8 inputs at most 6.6e-6.
+# The bound is 20x under GAP, the selection tolerance above, which therefore
+# never hides a logit error.
+LOGIT_ATOL = 1e-4
+# softmax of the kernel's own fp32 values: fp32 expf, sum and division
+OWN_SCORE_ATOL = 2e-6
+
+
+def logit_error(gpu_logits: np.ndarray, oracle_logits: np.ndarray) -> float:
+    """Largest |logit_gpu - logit_oracle| over every token and expert."""
+    g = np.asarray(gpu_logits, dtype=np.float64)
+    assert g.shape == oracle_logits.shape, (g.shape, oracle_logits.shape)
+    return float(np.max(np.abs(g - oracle_logits))) if g.size else 0.0
+
+
+def check_own_selection(gpu_scores: np.ndarray, gpu_ids: np.ndarray, gpu_logits: np.ndarray, label: str = "") -> int:
+    """The selection and softmax the kernel made from its own fp32 logits, exactly.
+
+    ids must be the first k of the (value descending, index ascending) order of
+    the row's fp32 logits -- a stable sort of the negated values, in which -0.0
+    and +0.0 compare equal -- and scores the softmax of those k values
+    (computed here in fp64) within OWN_SCORE_ATOL.  Returns the row count.
+    """
+    L = np.asarray(gpu_logits, dtype=np.float32)
+    ids = np.asarray(gpu_ids).astype(np.int64)
+    T, k = ids.shape
+    order = np.argsort(-L, axis=1, kind="stable")[:, :k]
+    bad = np.nonzero(np.any(order != ids, axis=1))[0]
+    assert bad.size == 0, (f"{label}: row {bad[0]} ids {ids[bad[0]]} are not the top-{k} of its own logits "
+                           f"{order[bad[0]]}")
+    v = np.take_along_axis(L, ids, axis=1).astype(np.float64)
+    e = np.exp(v - v[:, :1])
+    s = e / e.sum(axis=1, keepdims=True)
+    err = float(np.max(np.abs(s - np.asarray(gpu_scores, dtype=np.float64)))) if T else 0.0
+    assert err <= OWN_SCORE_ATOL, f"{label}: scores differ from the softmax of the selected logits by {err}"
+    return T

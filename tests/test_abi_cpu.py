@@ -207,3 +207,34 @@ def test_split_h_staging_slots_are_distinct(C, valid_rows):
             assert (owner, slot) not in seen
             seen.add((owner, slot))
     assert len(seen) == sum(n * C for n in n_own.values())
+
+
+def test_logits_entry_points_reject_before_cuda():
+    lib = tk.library()
+    f = lib.tk_gating_fused_topk_logits
+    assert f(16, 16, 8, 64, 16, 2, 16, 16, 0, 0) == tk.TK_ERR_INVALID_ARG      # null logits
+    assert f(16, 16, 8, 64, 16, 2, 16, 16, 20, 0) == tk.TK_ERR_ALIGNMENT       # logits not 16-byte aligned
+    assert f(16, 16, 8, 64, 20, 2, 16, 16, 0, 0) == tk.TK_ERR_UNSUPPORTED      # sizes are checked first
+    assert f(0, 16, 8, 64, 16, 2, 16, 16, 16, 0) == tk.TK_ERR_INVALID_ARG      # null hidden
+    assert f(0, 0, 0, 64, 16, 2, 0, 0, 0, 0) == tk.TK_OK                         # T == 0
+    g = lib.tk_gating_fused_topk_fp8_logits
+    assert g(16, 16, 16, 16, 8, 64, 16, 2, 16, 16, 0, 0) == tk.TK_ERR_INVALID_ARG
+    assert g(16, 16, 16, 16, 8, 64, 16, 2, 16, 16, 24, 0) == tk.TK_ERR_ALIGNMENT
+    assert g(16, 16, 16, 16, 8, 72, 16, 2, 16, 16, 0, 0) == tk.TK_ERR_UNSUPPORTED  # H % 16
+    assert g(0, 0, 0, 0, 0, 64, 16, 2, 0, 0, 0, 0) == tk.TK_OK
+
+
+def test_clock_counters_reject_null_pointers():
+    c = ctypes.c_uint64(0)
+    lib = tk.library()
+    assert lib.tk_gating_clock_counters(None, ctypes.byref(c), ctypes.byref(c), 0) == tk.TK_ERR_INVALID_ARG
+    assert lib.tk_gating_clock_counters(ctypes.byref(c), ctypes.byref(c), None, 1) == tk.TK_ERR_INVALID_ARG
+
+
+def test_binding_rejects_bad_logits_before_the_call():
+    from moe_router_gating_b200 import _binding
+    with pytest.raises(ValueError):
+        _binding._check_logits(torch.empty((3, 4)), 3, 5, torch.device("cpu"))
+    with pytest.raises(ValueError):
+        _binding._check_logits(torch.empty((3, 4), dtype=torch.float64), 3, 4, torch.device("cpu"))
+    _binding._check_logits(torch.empty((3, 4)), 3, 4, torch.device("cpu"))

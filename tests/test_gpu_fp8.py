@@ -3,7 +3,7 @@ tests/parity.py.  Inputs: the workloads' bf16 values quantized per token
 (hidden) and per expert (gate, expert-major) by torch on the CPU -- the same
 bits and scales feed both sides.  Covers split-H clusters and CTA pairs,
 half tiles, 512 experts, k up to 32, exact ties (duplicated experts quantize
-identically), the 65536 x 7168 launch on sampled rows, and a zero gate."""
+identically), the 65536 x 7168 launches on every row, and a zero gate."""
 import numpy as np
 import pytest
 import torch
@@ -57,12 +57,14 @@ def test_fp8_skew_ties():
     assert info["rows"] == workloads.SKEW.T
 
 
-def test_fp8_train_sampled_rows():
-    wl = workloads.TRAIN
-    rng = np.random.default_rng(3)
-    rows = np.unique(np.concatenate([np.arange(0, 256), np.arange(wl.T - 256, wl.T),
-                                     rng.choice(wl.T, 512, replace=False)]))
-    check_fp8(wl, rows=rows)
+def test_fp8_train_all_rows():
+    info = check_fp8(workloads.TRAIN)
+    assert info["rows"] == workloads.TRAIN.T
+
+
+def test_fp8_large_e_all_rows():
+    info = check_fp8(workloads.LARGE_E)
+    assert info["rows"] == workloads.LARGE_E.T
 
 
 def test_fp8_zero_gate_gives_uniform_scores():

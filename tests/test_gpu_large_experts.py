@@ -72,19 +72,18 @@ def test_ties_across_expert_groups(T):
     check_against_oracle(wl.hidden(), w, k, duplicate_pairs=pairs, label=f"gties_{T}")
 
 
-def test_large_e_workload_sampled_rows():
-    """The 65536 x 7168 x 512 launch the benchmark times; the oracle checks sampled rows."""
+def test_large_e_workload_all_rows():
+    """The 65536 x 7168 x 512 launch the benchmark times, every row against the oracle."""
     wl = workloads.LARGE_E
-    x_bits = wl.hidden()
-    w_bits = wl.gate_weight()
-    s, i = run_gpu(x_bits, w_bits, wl.k)
-    rng = np.random.default_rng(1)
-    rows = np.unique(np.concatenate([np.arange(0, 256), np.arange(wl.T - 256, wl.T),
-                                     rng.choice(wl.T, 512, replace=False)]))
-    ref = oracle.fused_topk_gating(x_bits[rows], w_bits, wl.k, want_logits=True)
-    parity.check(s, i, ref, rows=rows, label="large_e-sampled")
-    assert np.all((i >= 0) & (i < wl.E))
-    assert np.all(np.diff(s, axis=1) <= 0)
+    info = check_workload(wl)
+    assert info["rows"] == wl.T
+
+
+def test_e1024_workload_all_rows():
+    """65536 x 7168 x 1024: two expert groups per tile, every row against the oracle."""
+    wl = workloads.E1024
+    info = check_workload(wl)
+    assert info["rows"] == wl.T
 
 
 def test_large_k_workload():

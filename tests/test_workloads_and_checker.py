@@ -109,3 +109,30 @@ def test_checker_rejects_duplicate_order(case):
     ids[t, pa], ids[t, pb] = 21, 20
     with pytest.raises(AssertionError):
         parity.check(case.scores, ids, case, duplicate_pairs=((20, 21),))
+
+
+def test_own_selection_checker_accepts_the_rule_and_rejects_mistakes():
+    # ties resolve to the lower index, -0.0 equals +0.0
+    L = np.array([[0.5, 2.0, 2.0, -1.0, 0.0, -0.0],
+                  [-0.0, 0.0, -3.0, -0.0, 1.0, 1.0]], dtype=np.float32)
+    ids = np.array([[1, 2, 0, 4], [4, 5, 0, 1]], dtype=np.int32)
+    v = np.take_along_axis(L, ids, axis=1).astype(np.float64)
+    s = np.exp(v - v[:, :1]) / np.exp(v - v[:, :1]).sum(axis=1, keepdims=True)
+    assert parity.check_own_selection(s.astype(np.float32), ids, L) == 2
+    swapped = ids.copy()
+    swapped[0, :2] = [2, 1]                        # equal values in the wrong index order
+    with pytest.raises(AssertionError):
+        parity.check_own_selection(s.astype(np.float32), swapped, L)
+    zero_order = ids.copy()
+    zero_order[1, 2:] = [1, 0]                     # -0.0 and +0.0 are equal: index order decides
+    with pytest.raises(AssertionError):
+        parity.check_own_selection(s.astype(np.float32), zero_order, L)
+    with pytest.raises(AssertionError):            # a wrong score
+        parity.check_own_selection((s + 1e-4).astype(np.float32), ids, L)
+
+
+def test_logit_error_is_the_largest_difference():
+    a = np.zeros((3, 4))
+    b = a.copy()
+    b[2, 1] = -3e-5
+    assert parity.logit_error(b.astype(np.float32), a) == pytest.approx(3e-5, rel=1e-3)

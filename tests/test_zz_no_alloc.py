@@ -46,6 +46,7 @@ def test_static_scratch_back_to_back_on_one_stream():
     ref = [_call(tk.route_ptr, d, T, k, E)[1:] for d in (ids_a, ids_b)]
     outs = [_outputs(T, k, E) for _ in range(2)]
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())  # the sentinel fills and the ids land first
     for d, (off, ss, sp) in zip((ids_a, ids_b), outs):
         assert tk.route_static_ptr(d.data_ptr(), T, k, E, off.data_ptr(), ss.data_ptr(), sp.data_ptr(),
                                    s.cuda_stream) == tk.TK_OK
