@@ -341,6 +341,125 @@ TK_API tk_status tk_gating_route_plan(int64_t T, int32_t k, int32_t E, int32_t n
 TK_API tk_status tk_gating_route_static(const int32_t* ids, int64_t T, int32_t k, int32_t E, int32_t* offsets,
                                         int32_t* sorted_slots, int32_t* slot_pos, void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Expert-parallel dispatch and combine.
+ *
+ * The operation (chenxutan.com, "TileKernels 深度解析", section 4.2 "MoE
+ * Routing": fused_dispatch(tokens, expert_ids, num_experts, ep_group) sends
+ * every token to the GPUs holding the experts its expert_ids row names;
+ * fused_combine(expert_output, dispatch_indices, scores, ep_group) brings the
+ * experts' results back and sums them weighted by the gating scores).  In an
+ * expert-parallel group of R ranks, rank q holds experts [q*E/R, (q+1)*E/R).
+ * Rank q's receive buffer holds, for each of its experts in ascending order,
+ * for each source rank in ascending order, that source's rows for the expert
+ * in ascending assignment order s = t*k + j.  The expert outputs are expected
+ * in the same layout (one output row per received row).
+ *
+ * Both calls address the expert buffers through a device table of E row
+ * addresses: rows[e] = the address of this source rank's first row for
+ * expert e in the buffer of the rank that holds e (a local buffer, or another
+ * GPU's buffer opened with tk_gating_ep_ipc_open).  Assignment s with expert
+ * e = ids[s] at position p = slot_pos[s] of the expert-grouped order (offsets,
+ * sorted_slots, slot_pos from tk_gating_route) uses row rows[e] + (p -
+ * offsets[e]).  Dispatch stores each token row there; combine loads the
+ * expert output rows from there (the receiver pulls, as the page's section 6
+ * recommends), so the data crosses NVLink once and no all-to-all runs.
+ * Ordering between ranks is the caller's: every rank's dispatch has to be
+ * complete before the experts read the receive buffers, every expert output
+ * before combine reads it.  A row address that is not 16-byte aligned is
+ * skipped and sets bit 8 of the device error word (tk_gating_device_error).
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * tk_gating_fused_dispatch -- copy every placed assignment's token row to
+ * its row in the expert buffer.
+ *
+ *   tokens        device, bf16 [T, H] row-major, 16-byte aligned.
+ *   T, H, k, E    tokens (T >= 0), hidden size (H % 8 == 0), experts per
+ *                 token (1 <= k <= 32), experts (1 <= E <= 1024); T*k < 2^31.
+ *   ids           device, int32 [T, k]: the experts (tk_gating_fused_topk).
+ *   offsets       device, int32 [E + 1]     } tk_gating_route of ids
+ *   sorted_slots  device, int32 [T * k]     }
+ *   rows          device, uint64 [E]: destination address of expert e's first
+ *                 row for this rank (16-byte aligned; device or peer memory).
+ *   stream        cudaStream_t (void*), may be NULL.
+ *
+ * Errors: TK_ERR_INVALID_ARG (negative sizes, k or E < 1, null pointers when
+ * T > 0), TK_ERR_UNSUPPORTED (H % 8, k > 32, E > 1024, T*k >= 2^31),
+ * TK_ERR_ALIGNMENT (tokens not 16-byte, rows not 8-byte, the int32 arrays
+ * not 4-byte aligned), TK_ERR_CUDA (launch failure or no sm_100 device).
+ * T == 0 returns TK_OK and launches nothing.
+ */
+TK_API tk_status tk_gating_fused_dispatch(const void* tokens, int64_t T, int64_t H, int32_t k, int32_t E,
+                                          const int32_t* ids, const int32_t* offsets, const int32_t* sorted_slots,
+                                          const uint64_t* rows, void* stream);
+
+/*
+ * tk_gating_fused_combine -- out[t] = sum_j scores[t, j] * y(t, j), where
+ * y(t, j) is the expert output row of assignment (t, j), in fp32 (fused
+ * multiply-adds in rank order j = 0 .. k-1), rounded once to bf16.
+ * Assignments whose id is outside [0, E) or whose slot_pos is -1 contribute
+ * nothing.
+ *
+ *   rows          device, uint64 [E]: address of expert e's first output row
+ *                 for this rank (the table dispatch used, pointing into the
+ *                 expert output buffers).
+ *   ids, offsets  as tk_gating_fused_dispatch;  slot_pos  device, int32 [T, k]
+ *                 (tk_gating_route);  scores  device, fp32 [T, k].
+ *   out           device, out bf16 [T, H], 16-byte aligned.
+ *
+ * Errors as tk_gating_fused_dispatch (out 16-byte aligned, scores 4-byte).
+ */
+TK_API tk_status tk_gating_fused_combine(const uint64_t* rows, int64_t T, int64_t H, int32_t k, int32_t E,
+                                         const int32_t* ids, const int32_t* offsets, const int32_t* slot_pos,
+                                         const float* scores, void* out, void* stream);
+
+/*
+ * tk_gating_ep_rows_table -- the row-address tables of source rank `rank`
+ * from every rank's routing offsets (one small launch).
+ *
+ *   offsets_all   device, int32 [R, E + 1]: row s = rank s's tk_gating_route
+ *                 offsets (gathered from every rank); rank s has
+ *                 offsets_all[s, e+1] - offsets_all[s, e] assignments to e.
+ *   R, E, rank    ranks (E % R == 0, E <= 1024), this rank (0 <= rank < R).
+ *   bases         device, uint64 [R]: address of rank q's receive buffer, as
+ *                 this process sees it (its own, or opened from a handle).
+ *   out_bases     device, uint64 [R] or NULL: the same for the expert output
+ *                 buffers (rows of the same layout).
+ *   H             hidden size (row pitch H * 2 bytes).
+ *   rows          device, out uint64 [E]: tk_gating_fused_dispatch's table.
+ *   out_rows      device, out uint64 [E] or NULL: tk_gating_fused_combine's
+ *                 table (from out_bases).
+ *   recv_offsets  device, out int32 [E/R + 1]: the first row of each of this
+ *                 rank's experts in its own receive buffer (and the total).
+ *
+ * Errors: TK_ERR_INVALID_ARG (R < 1, rank outside [0, R), null pointers),
+ * TK_ERR_UNSUPPORTED (E % R != 0, E > 1024, H % 8), TK_ERR_ALIGNMENT,
+ * TK_ERR_CUDA.
+ */
+TK_API tk_status tk_gating_ep_rows_table(const int32_t* offsets_all, int32_t R, int32_t E, int32_t rank,
+                                         const uint64_t* bases, const uint64_t* out_bases, int64_t H, uint64_t* rows,
+                                         uint64_t* out_rows, int32_t* recv_offsets, void* stream);
+
+/*
+ * Inter-process handles of device buffers, so that a rank can address
+ * another rank's expert buffers (on another GPU over NVLink, or on the same
+ * GPU).  tk_gating_ep_ipc_handle writes a handle of TK_EP_IPC_HANDLE_BYTES
+ * bytes for the device pointer (the CUDA IPC handle of the allocation that
+ * contains it, plus the offset into it); another process passes those bytes to
+ * tk_gating_ep_ipc_open, which maps the allocation and returns the same
+ * buffer's address in that process; tk_gating_ep_ipc_close(ptr, handle) unmaps
+ * it.  The owner must keep the allocation alive while it is open elsewhere.
+ * TK_ERR_INVALID_ARG for null arguments or a pointer that is not device
+ * memory; TK_ERR_CUDA when the CUDA IPC call fails.
+ */
+#define TK_EP_IPC_HANDLE_BYTES 128
+TK_API tk_status tk_gating_ep_ipc_handle(const void* dev_ptr, void* handle);
+TK_API tk_status tk_gating_ep_ipc_open(const void* handle, void** dev_ptr);
+TK_API tk_status tk_gating_ep_ipc_close(void* dev_ptr, const void* handle);
+
 /* Static string for a status code. */
 TK_API const char* tk_gating_status_string(tk_status status);
 

@@ -346,6 +346,15 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
 
 }  // namespace
 
+namespace tkg {
+// The device error word of the current device for the other kernels of this
+// library (expert-parallel dispatch and combine); null without an sm_100 device.
+uint32_t* device_error_word() {
+  const DeviceState* d = device_state();
+  return d != nullptr && d->status == TK_OK ? d->err_word : nullptr;
+}
+}  // namespace tkg
+
 extern "C" {
 
 tk_status tk_gating_fused_topk(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,
