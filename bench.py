@@ -64,9 +64,10 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (profiling cases)")
     ap.add_argument("--precision", default="bf16", choices=("bf16", "fp8"),
                     help="bf16 (default) or FP8 E4M3 inputs with per-token / per-expert scales")
-    ap.add_argument("--op", default="gating", choices=("gating", "route", "gating_route"),
+    ap.add_argument("--op", default="gating", choices=("gating", "route", "gating_route", "ep"),
                     help="gating (default); route: routing metadata of the workload's T x k ids; "
-                         "gating_route: both, chained on the device")
+                         "gating_route: both, chained on the device; ep: expert-parallel dispatch and combine "
+                         "of the workload's tokens (one rank)")
     return ap.parse_args()
 
 
@@ -301,18 +302,29 @@ def run_ours(args, wl):
         wqd, wsd = torch.from_numpy(wq).to(dev), torch.from_numpy(ws).to(dev)
         hidden_bytes = wl.T * wl.H + 4 * wl.T
 
-        def step():
-            tk.fused_topk_gating_fp8(x, xsd, wqd, wsd, wl.k, scores=scores, ids=ids, stream=stream)
+        def gate(xx):
+            return lambda: tk.fused_topk_gating_fp8(xx, xsd, wqd, wsd, wl.k, scores=scores, ids=ids, stream=stream)
     else:
         x_host = workloads.to_torch_bf16(rank_wl.hidden())
         w = workloads.to_torch_bf16(rank_wl.gate_weight()).to(dev)
         x = x_host.to(dev)
         hidden_bytes = wl.T * wl.H * 2
 
-        def step():
-            tk.fused_topk_gating(x, w, wl.k, scores=scores, ids=ids, stream=stream)
+        def gate(xx):
+            return lambda: tk.fused_topk_gating(xx, w, wl.k, scores=scores, ids=ids, stream=stream)
     big = hidden_bytes > L2_BYTES
-    flush = None if big else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    # 16 MB up to L2: back-to-back launches over rotating hidden buffers that together
+    # exceed twice L2 (each launch reads a hidden tensor evicted since its last use)
+    rotate = not big and hidden_bytes >= 16 * 1024 * 1024
+    n_buf = max(4, -(-2 * L2_BYTES // hidden_bytes) + 1) if rotate else 1
+    xs_dev = [x] + [x.clone() for _ in range(n_buf - 1)]
+    steps_of = [gate(xx) for xx in xs_dev]
+    step_count = [0]
+
+    def step():
+        steps_of[step_count[0] % n_buf]()
+        step_count[0] += 1
+    flush = None if big or rotate else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -324,8 +336,8 @@ def run_ours(args, wl):
     torch.cuda.synchronize(dev)
     tk.clock_counters(clear=True)
     with sampler:
-        if big:
-            # inputs larger than L2: back-to-back launches between two events
+        if big or rotate:
+            # inputs larger than L2 (or rotating buffers): back-to-back launches between two events
             ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             ev0.record(stream)
             for _ in range(args.steps):
@@ -429,6 +441,8 @@ def run_ours(args, wl):
             "precision": args.precision,
             "l2": ("inputs larger than L2: hidden is %.0f MB per step (gate %.2f MB stays L2-resident by design)"
                    % (hidden_bytes / 1e6, wl.H * wl.E * 2 / 1e6)) if big else
+                  ("back-to-back launches over %d hidden buffers (%.0f MB together, more than twice L2); the gate "
+                   "stays L2-resident by design" % (n_buf, n_buf * hidden_bytes / 1e6)) if rotate else
                   "L2 flushed (256 MB write) before every timed launch; each launch timed alone",
             "parallelism": "single GPU" if world == 1 else f"{world} ranks, independent token shards, no collective",
             "launch": plan,
@@ -543,7 +557,30 @@ def oracle_single_thread_rate(wl, seconds: float):
     return v, rows, dt
 
 
+def time_rotating(steps_of, stream, steps: int) -> float:
+    """Mean ms per call of back-to-back calls that cycle through distinct input
+    buffers (steps_of[i] gates buffer i): each call reads a hidden tensor that
+    the calls since its last use have evicted from L2."""
+    import torch
+    for st in steps_of:
+        st()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        steps_of[i % len(steps_of)]()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
 def per_workload_summary(dev, peaks, peak_src, cpu_seconds: float, with_cpu: bool) -> dict:
+    """Every router workload on one GPU.  Timing: inputs larger than L2 back to
+    back; inputs of 16 MB up to L2 back to back over rotating hidden buffers
+    (together more than twice L2; the gate stays L2-resident by design);
+    smaller ones one call at a time after an L2 flush.  Each entry also gives
+    the one-call-after-a-flush time (which carries the ~5 us launch latency
+    after the flush kernel) and the kernel's own span measured in the kernel."""
     import torch
 
     import moe_router_gating_b200 as tk
@@ -552,23 +589,42 @@ def per_workload_summary(dev, peaks, peak_src, cpu_seconds: float, with_cpu: boo
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     for name in SUMMARY_WORKLOADS:
         wl = workloads.WORKLOADS[name]
+        hidden_bytes = wl.T * wl.H * 2
         x = workloads.to_torch_bf16(wl.hidden()).to(dev)
         w = workloads.to_torch_bf16(wl.gate_weight()).to(dev)
         s = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
         i = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
-        big = wl.T * wl.H * 2 > L2_BYTES
+        big = hidden_bytes > L2_BYTES
+        rotate = not big and hidden_bytes >= 16 * 1024 * 1024
 
-        def step():
-            tk.fused_topk_gating(x, w, wl.k, scores=s, ids=i, stream=stream)
-        tk.clock_counters(clear=True)
-        steps = 20 if big else 200
-        ms = time_calls(step, stream, steps, None if big else flush)
+        def gate(xx):
+            return lambda: tk.fused_topk_gating(xx, w, wl.k, scores=s, ids=i, stream=stream)
+        flushed_ms = None
+        if not big:
+            tk.clock_counters(clear=True)
+            flushed_ms = time_calls(gate(x), stream, 200, flush)
         clk = tk.clock_counters(clear=True)
+        if big:
+            ms = time_calls(gate(x), stream, 20, None)
+            clk = tk.clock_counters(clear=True)
+            timing = "back-to-back calls, inputs larger than L2"
+        elif rotate:
+            n = max(4, -(-2 * L2_BYTES // hidden_bytes) + 1)
+            xs = [x] + [x.clone() for _ in range(n - 1)]
+            ms = time_rotating([gate(xx) for xx in xs], stream, 20 * n)
+            clk = tk.clock_counters(clear=True)
+            timing = (f"back-to-back calls over {n} hidden buffers ({n * hidden_bytes / 1e6:.0f} MB, more than "
+                      "twice L2); the gate stays L2-resident")
+            del xs
+        else:
+            ms = flushed_ms
+            timing = "each call alone after an L2 flush (256 MB write), mean of 200"
         roof = roofline_of(wl, ms, False, peaks, peak_src)
+        launches = clk["launches"] or 1
         entry = {"T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "us_per_call": ms * 1e3,
-                 "tokens_per_s": wl.T / (ms / 1e3),
-                 "timing": ("back-to-back calls, inputs larger than L2" if big else
-                            "each call alone after an L2 flush (256 MB write), mean of %d" % steps),
+                 "tokens_per_s": wl.T / (ms / 1e3), "timing": timing,
+                 "us_per_call_after_flush": flushed_ms * 1e3 if flushed_ms is not None else None,
+                 "kernel_span_us_in_kernel": clk["elapsed_ns"] / launches / 1e3 if clk["launches"] else None,
                  "roofline": {"bound": roof["bound"], "frac": roof["frac"], "roofline_frac": roof["roofline_frac"],
                               "roofline_frac_sustained": roof["roofline_frac_sustained"],
                               "roofline_us": roof["roofline_us"]},
@@ -723,6 +779,87 @@ def run_route_ours(args, wl):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# expert-parallel dispatch and combine (--op ep), one GPU, one rank
+# ---------------------------------------------------------------------------
+EP_METRIC = "expert-parallel dispatch + combine tokens/s"
+
+
+def run_ep_ours(args, wl):
+    """Dispatch copies every placed assignment's token row to its expert row;
+    combine sums each token's k expert rows.  One rank, so every row stays in
+    this GPU's memory; each kernel is timed on its own (CUDA events, inputs
+    larger than L2 at the 4096-token shape: T*k rows of 14 KB = 470 MB)."""
+    import torch
+
+    import moe_router_gating_b200 as tk
+    from moe_router_gating_b200 import ep
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T, H, E, k = wl.T, wl.H, wl.E, wl.k
+    stream = torch.cuda.current_stream(dev)
+    x = workloads.to_torch_bf16(wl.hidden()).to(dev)
+    ids = torch.from_numpy(workloads.expert_ids(T, k, E, seed=0, kind="skew")).to(dev)
+    scores = torch.rand((T, k), dtype=torch.float32, device=dev)
+    g = ep.ExpertParallelGroup(E, H, capacity=T * k, device=dev)
+    offsets, sorted_slots, slot_pos = tk.route(ids, E)
+    rows, out_rows, recv_offsets = ep.rows_table(offsets.view(1, E + 1), 0, g.bases, g.out_bases, H)
+    g.output.copy_(g.recv)  # experts = identity for the timing
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+
+    def dispatch():
+        ep.dispatch_rows(x, ids, offsets, sorted_slots, rows, E, stream)
+
+    def combine():
+        ep.combine_rows(out_rows, ids, offsets, slot_pos, scores, out, E, stream)
+
+    def timed(fn, steps):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / steps
+
+    tk.device_error(clear=True)
+    sampler = ClockSampler(0)
+    with sampler:
+        t_d = timed(dispatch, args.steps)
+        t_c = timed(combine, args.steps)
+    if tk.device_error(clear=True):
+        raise SystemExit("an expert-parallel kernel reported a bad row address")
+    placed = T * k
+    d_bytes = 2 * (2 * H) * placed            # each placed row read once (from L2 when repeated) and written once
+    c_bytes = (2 * H) * placed + 2 * H * T + 12 * T * k   # k rows read per token, one row written, metadata
+    peaks, peak_src = load_peaks()
+    ms = t_d + t_c
+    line = {
+        "metric": EP_METRIC, "value": T / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{wl.name}-shaped tokens: T={T} H={H} E={E} k={k}, skewed seeded ids, one rank",
+                   "l2": "dispatch writes and combine reads 470 MB of expert rows per step (more than L2)"},
+        "roofline": {"bound": "hbm", "dispatch_us": t_d * 1e3, "combine_us": t_c * 1e3,
+                     "dispatch_gbs": d_bytes / (t_d / 1e3) / 1e9, "combine_gbs": c_bytes / (t_c / 1e3) / 1e9,
+                     "dispatch_frac": d_bytes / (t_d / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "combine_frac": c_bytes / (t_c / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": f"{peak_src}; copy GB/s",
+                     "algorithmic_bytes": {"dispatch": d_bytes, "combine": c_bytes}},
+        "gpu_launches": args.steps * 2,
+        "clocks": sampler.summary(),
+        "note": "one rank: every row stays local; across GPUs the same stores and loads go to peer memory "
+                "(not measured: one GPU per call on this pool)",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     wl = workloads.WORKLOADS[args.workload]
@@ -732,6 +869,8 @@ def main():
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers --op gating only"}))
             return 0
+        if args.op == "ep":
+            return run_ep_ours(args, wl)
         return run_route_ours(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)

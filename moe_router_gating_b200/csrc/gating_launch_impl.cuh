@@ -36,18 +36,22 @@ template <int KMAX, int CG, bool FP8, int EG>
 tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
                            const CUtensorMap& mw, const RowTileParams& prm, cudaStream_t stream) {
   auto kernel = gating_row_tiles_kernel<KMAX, CG, FP8, EG>;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CG;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: CTAs may start on SMs the previous kernel has
+  // left and set up while it finishes (the producer waits before its loads)
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CG;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(pl.threads);
   cfg.dynamicSmemBytes = pl.smem_bytes;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = CG > 1 ? 1 : 0;
+  cfg.numAttrs = CG > 1 ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, kernel, mx, mx64, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
   return TK_OK;
 }
@@ -56,18 +60,20 @@ template <int KMAX, int C, bool FP8>
 tk_status launch_split_h_c(const tk_gating_plan& plan, const CUtensorMap& mx, const CUtensorMap& mw,
                            const SplitHParams& prm, cudaStream_t stream) {
   auto kernel = gating_split_h_kernel<KMAX, C, FP8>;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // as launch_row_tiles
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.num_tiles * C);
   cfg.blockDim = dim3(plan.threads);
   cfg.dynamicSmemBytes = plan.smem_bytes;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kernel, mx, mw, prm) != cudaSuccess) return TK_ERR_CUDA;
   return TK_OK;
 }

@@ -313,6 +313,10 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
+      // The launch may overlap the previous kernel's tail (programmatic dependent
+      // launch): every global read and write of this kernel follows this wait,
+      // the later ones through the ring's and accumulator's barriers.
+      griddep_wait();
       const uint64_t pol_x = l2_policy_evict_first();  // hidden: streamed once
       const uint64_t pol_w = l2_policy_evict_last();   // gate: re-read by every tile
       // gate box j of a K slice starts at column j * 64 + (j < bpc0 ? col_a : col_b): this

@@ -8,22 +8,25 @@
 //
 //   1. mainloop (as in the row-tile kernel, one tile, k-blocks [kb0, kb1)):
 //      partial_r[128, E] in tensor memory;
-//   2. cluster barrier: every CTA's ring is drained, so its shared memory can
-//      take the exchange;
-//   3. CTA r owns the tile rows t with t % C == r.  Every CTA pushes row t of its
-//      partial (tensor memory -> registers -> distributed shared memory stores)
-//      into slot [t / C][r] of the owner's staging area;
-//   4. cluster barrier: the staging areas are complete;
-//   5. each owned row is split into G column segments, one thread each: the
-//      thread adds the C partials of its segment from local shared memory in
-//      rank order 0..C-1 (so a logit does not depend on which CTA owns its
-//      row), keeps a top-k of the segment, and the G lists are merged with warp
-//      shuffles; then softmax and store.
+//   2. once its own ring is idle, every CTA copies its partial rows from tensor
+//      memory into its own shared memory (local stores only);
+//   3. cluster barrier: every CTA's partial rows are visible to the cluster;
+//   4. CTA r owns the tile rows t with t % C == r.  Each owned row is split
+//      into G column segments, one thread each: the thread reads the C
+//      partials of its segment -- its own from local shared memory, the others
+//      straight from the other CTAs' shared memory (distributed shared memory
+//      loads: the owner pulls) -- adds them in rank order 0..C-1 (so a logit
+//      does not depend on which CTA owns its row), keeps a top-k of the
+//      segment, and the G lists are merged with warp shuffles; then softmax
+//      and store;
+//   5. cluster barrier: no CTA reuses or releases its shared memory while an
+//      owner may still read it.
 //
 // More than 256 experts (up to 512): one MMA per chunk of at most 256 experts
-// and K step (chunk c in tensor-memory columns from 256c), and steps 2..5 run
-// once per 256-expert column range: each pass pushes and reduces its columns
-// and the owners keep their running top-k lists across passes.  More than 512
+// and K step (chunk c in tensor-memory columns from 256c), and steps 2..4 run
+// once per 256-expert column range (with a cluster barrier between passes):
+// each pass stages and reduces its columns and the owners keep their running
+// top-k lists across passes.  More than 512
 // (up to 1024): steps 1..5 run once per group of 512 experts, the ring position
 // carried over; the owners' lists run over both groups.
 //
@@ -45,13 +48,11 @@
 
 namespace tkg {
 
-// Warps: 0 producer, 1 MMA, 2..5 push partial rows (TMEM lane quadrants), 6..7
+// Warps: 0 producer, 1 MMA, 2..5 stage partial rows (TMEM lane quadrants), 6..7
 // join the reduction; all 8 reduce.
 constexpr int SPLIT_THREADS = 256;
 constexpr int SPLIT_WARPS = SPLIT_THREADS / 32;
 constexpr int PUSH_WARPS = 4;
-constexpr int PUSH_SCRATCH_STRIDE = 36;                            // floats per scratch row (bank spread)
-constexpr int PUSH_SCRATCH_BYTES = 32 * PUSH_SCRATCH_STRIDE * 4;   // one 32 x 32 chunk per push warp
 
 struct SplitHParams {
   int32_t T, H, E, k;
@@ -86,8 +87,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + p.stages * p.kps * A_STAGE_BYTES;
   float* staging = reinterpret_cast<float*>(smem);  // reuses the ring once every CTA's MMAs are done
-  float* scratch = reinterpret_cast<float*>(sB + p.stages * p.kps * p.b_boxes * B_BOX_BYTES);  // after the ring
-  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scratch) + PUSH_WARPS * PUSH_SCRATCH_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + p.stages * p.kps * p.b_boxes * B_BOX_BYTES);  // after the ring
   uint64_t* empty = full + p.stages;
   uint64_t* acc_full = empty + p.stages;
   uint64_t* drain = acc_full + 1;
@@ -119,6 +119,9 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     tmem_alloc(tmem_holder, p.tmem_cols);
     tmem_relinquish();
   }
+  // The launch may overlap the previous kernel's tail (programmatic dependent
+  // launch); the set-up above touches no global memory, everything below may.
+  griddep_wait();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -245,8 +248,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
       __syncwarp();
     }
 
-    // Epilogue warps wait for this CTA's accumulator; then all rings of the
-    // cluster are idle and may be overwritten by the exchange.
+    // The staging warps wait for this CTA's accumulator.
     const bool push_warp = warp >= 2 && warp < 2 + PUSH_WARPS;
     bool acc_ok = true;
     if (push_warp) {
@@ -254,83 +256,82 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
       acc_ok = __all_sync(0xffffffffu, acc_ok && *abort_flag == 0);
     }
 
+    // This CTA's ring is idle once its producer has drained its loads and its
+    // MMAs are done (the push warps waited for acc_full): the partial rows may
+    // overwrite it.
+    __syncthreads();
+
     for (int pass = 0; pass < n_chunks; ++pass) {
       const int col0 = pass * N_CHUNK;                        // first TMEM column of this pass
       const int pass_cols = min(N_CHUNK, p.E - (e0 + col0));  // experts e0 + col0 .. of this pass
-      // every ring (first pass) or every staging area (later passes) is free
-      tc_fence_before_sync();
-      cluster_arrive_release();
-      cluster_wait_acquire();
-      tc_fence_after_sync();
+      // the previous pass's partials have been pulled by every owner
+      if (pass > 0) {
+        cluster_arrive_release();
+        cluster_wait_acquire();
+      }
 
-      // ---------------- push partial rows to their owners ----------------
-      // Each 32-row x 32-column chunk (row per thread from tensor memory) is
-      // transposed through this warp's scratch so that every remote store writes 128
-      // contiguous bytes of one row: 8 lanes per row, 4 rows per store instruction.
+      // ---------------- partial rows into this CTA's own shared memory ----------------
+      // Thread = tile row (tensor-memory lane), 32 columns per load; each thread
+      // stores its row's 128 contiguous bytes (rows 260 floats apart: the eight
+      // lanes of a quarter warp hit 32 distinct banks).
       if (push_warp) {
         const int quad = warp & 3;
         if (acc_ok && quad * 32 < valid_rows) {
           const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
-          float* my_scratch = scratch + (warp - 2) * (PUSH_SCRATCH_BYTES / 4);
-          const int sub_row = lane >> 3;       // 0..3: row within a group of 4
-          const int col4 = (lane & 7) * 4;     // column offset within the chunk
-          // 64 columns per tensor-memory round trip, pushed as two 32-column chunks
+          const int t = quad * 32 + lane;  // tile-local row of this thread
+          float* row = staging + static_cast<size_t>(t) * p.row_stride;
+          // 64 columns per tensor-memory round trip
           for (int c0 = 0; c0 < pass_cols; c0 += 64) {
             uint32_t v[2][32];
             const bool second = c0 + 32 < pass_cols;  // warp-uniform
             tmem_ld_32(lane_base + c0, v[0]);
             if (second) tmem_ld_32(lane_base + c0 + 32, v[1]);
             tmem_ld_wait();
+            if (t < valid_rows) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (h == 1 && !second) break;
-              const int cc = c0 + 32 * h;
+              for (int h = 0; h < 2; ++h) {
+                if (h == 1 && !second) break;
 #pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(my_scratch + lane * PUSH_SCRATCH_STRIDE + j) =
-                    make_float4(__uint_as_float(v[h][j]), __uint_as_float(v[h][j + 1]), __uint_as_float(v[h][j + 2]),
-                                __uint_as_float(v[h][j + 3]));
-              __syncwarp();
-#pragma unroll
-              for (int rr = 0; rr < 32; rr += 4) {
-                const int t = quad * 32 + rr + sub_row;  // tile-local row
-                if (t < valid_rows && cc + col4 < pass_cols) {
-                  const float4 val =
-                      *reinterpret_cast<const float4*>(my_scratch + (rr + sub_row) * PUSH_SCRATCH_STRIDE + col4);
-                  float* dst =
-                      staging + static_cast<size_t>((t / C) * C + static_cast<int>(r)) * p.row_stride + cc + col4;
-                  const unsigned owner = static_cast<unsigned>(t % C);
-                  float* target = owner == r ? dst : static_cast<float*>(__cluster_map_shared_rank(dst, owner));
-                  *reinterpret_cast<float4*>(target) = val;
-                }
+                for (int j = 0; j < 32; j += 4)
+                  *reinterpret_cast<float4*>(row + c0 + 32 * h + j) =
+                      make_float4(__uint_as_float(v[h][j]), __uint_as_float(v[h][j + 1]),
+                                  __uint_as_float(v[h][j + 2]), __uint_as_float(v[h][j + 3]));
               }
-              __syncwarp();
             }
           }
         }
       }
       tc_fence_before_sync();
-      cluster_arrive_release();  // every owner's staging area is complete past this point
+      cluster_arrive_release();  // every CTA's partial rows are visible to the cluster past this point
       cluster_wait_acquire();
       if (warp == 1 && eg + 1 == p.e_groups && pass + 1 == n_chunks) {  // all tensor-memory reads are done
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, p.tmem_cols);
       }
 
-      // ---------------- reduce owned rows of this pass into the running top-k ----------------
+      // ---------------- owners pull their rows' partials and reduce ----------------
+      // Owner r's row t (t % C == r) sums partial_q[t] over q = 0 .. C-1 in rank
+      // order (so a logit does not depend on which CTA owns its row), reading the
+      // other CTAs' shared memory directly (distributed shared memory loads).
       if (active) {
+        const int t_own = static_cast<int>(r) + C * slot;
         float hs = 1.0f;  // FP8: the row's token scale
-        if constexpr (FP8) hs = __ldg(p.hscale + static_cast<int64_t>(tile) * BLOCK_M + static_cast<int>(r) + C * slot);
-        // segment `seg` takes every group-th float4 of the row: consecutive lanes
-        // read consecutive 16-byte words (no bank conflicts), and each thread still
-        // offers its columns in increasing order
-        const float* rows = staging + static_cast<size_t>(slot) * C * p.row_stride;
+        if constexpr (FP8) hs = __ldg(p.hscale + static_cast<int64_t>(tile) * BLOCK_M + t_own);
+        const float* mine = staging + static_cast<size_t>(t_own) * p.row_stride;
+        const uint32_t mine_addr = smem_u32(mine);
+        uint32_t peer[C];
+#pragma unroll
+        for (int q = 0; q < C; ++q) peer[q] = map_shared_rank(mine_addr, static_cast<uint32_t>(q));
         const int ebase = e0 + col0;
-        // the summed (and, FP8, scaled) logits of columns c .. c+3 of this row
+        // segment `seg` takes every group-th float4 of the row: consecutive lanes
+        // read consecutive 16-byte words, and each thread still offers its
+        // columns in increasing order
         auto column_quad = [&](int c) {
           float4 v[C];
 #pragma unroll
-          for (int q = 0; q < C; ++q) v[q] = *reinterpret_cast<const float4*>(rows + q * p.row_stride + c);
+          for (int q = 0; q < C; ++q)
+            v[q] = q == static_cast<int>(r) ? *reinterpret_cast<const float4*>(mine + c)
+                                              : ld_shared_cluster_f4(peer[q] + static_cast<uint32_t>(c) * 4u);
           float4 acc = v[0];
 #pragma unroll
           for (int q = 1; q < C; ++q) {  // rank order: the same sum whichever CTA owns the row
@@ -349,8 +350,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
           return acc;
         };
         float* dump = p.logits == nullptr ? nullptr
-                                          : p.logits + (static_cast<int64_t>(tile) * BLOCK_M + static_cast<int>(r) +
-                                                        C * slot) * p.E + ebase;
+                                          : p.logits + (static_cast<int64_t>(tile) * BLOCK_M + t_own) * p.E + ebase;
         for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
           const float4 acc = column_quad(c);
           if (dump != nullptr) {
@@ -366,9 +366,10 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
         }
       }
     }
-    // the next expert group's loads overwrite this CTA's staging area: every
-    // owner of this CTA has read it
-    if (eg + 1 < p.e_groups) __syncthreads();
+    // every owner has pulled its rows from this CTA: its shared memory may take
+    // the next expert group's loads, or be released when the CTA exits
+    cluster_arrive_release();
+    cluster_wait_acquire();
   }
 
   // ---------------- merge the segments, softmax, store ----------------

@@ -112,16 +112,18 @@ tk_status launch_scatter(const tk_route_plan& pl, const tkg::RouteParams& p, cud
   cfg.blockDim = dim3(pl.threads);
   cfg.dynamicSmemBytes = pl.scatter_smem_bytes;
   cfg.stream = stream;
-  if (pl.ctas == 1)
-    return cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, true>, p) == cudaSuccess ? TK_OK : TK_ERR_CUDA;
-  // programmatic dependent launch: the scatter kernel may start once every
-  // count CTA has started; it waits (griddepcontrol.wait) for the count
+  // programmatic dependent launch.  One CTA: the kernel may start while the
+  // previous kernel (typically the gating) finishes, and waits for it before
+  // reading ids.  Several: the scatter kernel may start once every count CTA has
+  // passed its own dependency wait; it waits (griddepcontrol.wait) for the count
   // kernel's completion before reading the counts table
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (pl.ctas == 1)
+    return cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, true>, p) == cudaSuccess ? TK_OK : TK_ERR_CUDA;
   return cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, false>, p) == cudaSuccess ? TK_OK : TK_ERR_CUDA;
 }
 
@@ -148,6 +150,11 @@ tk_status launch_route(const tk_route_plan& pl, const int32_t* ids, int64_t n, i
     cfg.blockDim = dim3(pl.threads);
     cfg.dynamicSmemBytes = pl.count_smem_bytes;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];  // a programmatic dependent of the previous kernel (see route_count_kernel)
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, tkg::route_count_kernel, p) != cudaSuccess) return TK_ERR_CUDA;
   }
   if (E <= 16) return launch_scatter<4>(pl, p, stream);

@@ -111,6 +111,9 @@ __device__ __forceinline__ void route_cta_warp_counts(const RouteParams& p, int3
 
 // Dynamic shared memory: hist[ROUTE_WARPS][Ep] int32.
 __global__ void __launch_bounds__(ROUTE_THREADS) route_count_kernel(const RouteParams p) {
+  // launched as a programmatic dependent of whatever precedes it (the gating
+  // kernel, typically): the ids are complete and visible past this wait
+  pdl_wait_primary();
   pdl_launch_dependents();  // the scatter kernel may start its own recount now
   extern __shared__ int32_t route_smem[];
   int64_t beg, end;
@@ -230,8 +233,11 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31u;
 
-  // 1. this CTA's per-warp counts (the ids were complete before the count
-  //    kernel started, so they may be read before the dependency wait)
+  // 1. this CTA's per-warp counts.  One CTA: this kernel is the programmatic
+  //    dependent of whatever precedes it and waits for it first.  Several: the
+  //    count kernel let this one start only after its own wait, so the ids are
+  //    complete and may be read before this kernel's dependency wait.
+  if (SINGLE) pdl_wait_primary();
   int64_t beg, end;
   route_warp_range(p, &beg, &end);
   route_cta_warp_counts(p, base, beg, end);

@@ -58,6 +58,10 @@ __device__ __forceinline__ void record_launch_clock(uint64_t* clock, uint64_t t0
   atomicAdd(c + 2, 1ull);
 }
 
+// Programmatic dependent launch: wait until the grids this one depends on have
+// completed and their memory is visible (returns at once for a plain launch).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t lane_id() {
   uint32_t l;
   asm volatile("mov.u32 %0, %%laneid;" : "=r"(l));

@@ -57,8 +57,7 @@ tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* p
   const int kps = g_pad > tkg::N_CHUNK ? 1 : tkg::KB_PER_STAGE;   // a slice of 512 experts is 80 KB
   const int b_boxes = (g_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES;
-  const int scratch = tkg::PUSH_WARPS * tkg::PUSH_SCRATCH_BYTES;
-  int stages = (kMaxDynamicSmem - kSmemReserve - scratch) / (kps * stage_bytes);
+  int stages = (kMaxDynamicSmem - kSmemReserve) / (kps * stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   const int row_stride = split_row_stride(E);
   // the staged partial rows of a tile (one 256-expert pass at a time) reuse the ring
@@ -74,7 +73,7 @@ tk_status plan_split_h(int64_t T, int64_t H, int64_t E, int C, tk_gating_plan* p
   plan->grid = static_cast<int32_t>(tiles * C);
   plan->cluster = C;
   plan->threads = tkg::SPLIT_THREADS;
-  plan->smem_bytes = stages * kps * stage_bytes + scratch + kSmemReserve;
+  plan->smem_bytes = stages * kps * stage_bytes + kSmemReserve;
   plan->tmem_cols = static_cast<int32_t>(pow2_at_least(round_up(g_pad, 32)));
   plan->slices_per_stage = kps;
   plan->expert_groups = n_pad > tkg::E_GROUP ? 2 : 1;
