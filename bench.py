@@ -720,6 +720,18 @@ def run_route_ours(args, wl):
     elapsed_ms = sum(per)
     ms_per_step = elapsed_ms / args.steps
     value = T * args.steps / (elapsed_ms / 1e3)
+    gating_alone_ms = None
+    if chain:
+        # the gating call alone, timed the same way in the same run: the routing's added cost
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        gating_alone_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
 
     # end to end: pinned host ids -> device, route, the three outputs -> pinned host
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
@@ -761,6 +773,9 @@ def run_route_ours(args, wl):
         "gpu_launches": args.steps * (3 if chain else 2),
         "clocks": sampler.summary(),
     }
+    if chain:
+        line["gating_alone_ms_per_step"] = gating_alone_ms
+        line["routing_added_us"] = (ms_per_step - gating_alone_ms) * 1e3
     if not chain:
         ach = bytes_alg / (ms_per_step / 1e3) / 1e9
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -148,8 +148,8 @@ def test_plan_large_expert_counts():
     assert p["variant"] == 3 and p["n_pad"] == 384 and p["tmem_cols"] == 512
     p = tk.make_plan(4096, 7168, 512, 32, 148)      # split-H, one 80 KB K slice per stage
     assert p["variant"] == 2 and p["slices_per_stage"] == 1 and p["tmem_cols"] == 512
-    p = tk.make_plan(4096, 7168, 256, 8, 148)
-    assert p["slices_per_stage"] == 2
+    p = tk.make_plan(4096, 7168, 256, 8, 148)      # split-H: one K slice per ring stage
+    assert p["slices_per_stage"] == 1 and p["stages"] == 4
     p = tk.make_plan(65536, 7168, 1024, 8, 148)     # two expert groups of 512, one after the other
     assert p["variant"] == 3 and p["n_pad"] == 1024 and p["expert_groups"] == 2 and p["tmem_cols"] == 512
     p = tk.make_plan(1, 7168, 1000, 8, 148)
@@ -238,3 +238,4 @@ def test_binding_rejects_bad_logits_before_the_call():
     with pytest.raises(ValueError):
         _binding._check_logits(torch.empty((3, 4), dtype=torch.float64), 3, 4, torch.device("cpu"))
     _binding._check_logits(torch.empty((3, 4)), 3, 4, torch.device("cpu"))
+

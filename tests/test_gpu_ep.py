@@ -83,6 +83,19 @@ def run_case(R, T, H, k, E, seed, kind="uniform"):
     routes = [tk.route(d, E) for d in d_ids]
     offsets_all = torch.stack([r[0] for r in routes])
     tables = [ep.rows_table(offsets_all, s, bases, out_bases, H) for s in range(R)]
+    # the device tables against the host plan of the same counts
+    counts = np.diff(offsets_all.cpu().numpy().astype(np.int64), axis=1)
+    base_list = bases.cpu().numpy().astype(np.uint64)
+    out_list = out_bases.cpu().numpy().astype(np.uint64)
+    for s in range(R):
+        plan = ep.exchange_plan(counts, s)
+        per = E // R
+        rows = tables[s][0].cpu().numpy().astype(np.uint64)
+        orows = tables[s][1].cpu().numpy().astype(np.uint64)
+        for e in range(E):
+            q = e // per
+            assert int(rows[e]) == int(base_list[q]) + plan.dest_row[e] * 2 * H, (s, e)
+            assert int(orows[e]) == int(out_list[q]) + plan.dest_row[e] * 2 * H, (s, e)
     for s in range(R):  # every source rank's dispatch writes into every receive buffer
         x = bf16_bits_to_torch(toks[s]).to(dev)
         ep.dispatch_rows(x, d_ids[s], routes[s][0], routes[s][1], tables[s][0], E)

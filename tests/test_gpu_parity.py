@@ -81,6 +81,8 @@ def test_train_workload_all_rows():
     (20000, 256, 256, 8), (19000, 128, 40, 3), (10000, 7168, 256, 8), (100, 7168, 256, 16), (3, 2048, 64, 4),
     # CTA pairs with a balanced last round of 128-token tiles (E padding in the upper expert half)
     (19999, 512, 200, 8), (60000, 512, 136, 16), (18945, 1024, 256, 1),
+    # one CTA per tile, E <= 64, a partly filled last round
+    (9473, 256, 64, 8), (12345, 512, 48, 5), (38000, 256, 56, 6),
 ])
 def test_ragged_shapes(T, H, E, k):
     wl = workloads.RouterWorkload(f"shape_{T}_{H}_{E}_{k}", T, H, E, k, seed=3)
@@ -160,3 +162,26 @@ def test_host_entry_point_matches_device_entry_point():
     torch.cuda.synchronize()
     s_ref, i_ref = tk.fused_topk_gating(xb.cuda(), w, wl.k)
     assert torch.equal(i_h, i_ref.cpu()) and torch.equal(s_h, s_ref.cpu())
+
+
+def test_gating_right_after_a_kernel_that_writes_hidden():
+    """The gating kernels are launched as programmatic dependents of the previous
+    kernel: their loads must still see what that kernel wrote (here a large copy
+    into the hidden buffer, issued just before each gating call on the stream)."""
+    for wl in (workloads.RouterWorkload("pdl_pairs", 20000, 1024, 256, 8, seed=21),
+               workloads.RouterWorkload("pdl_split", 300, 7168, 256, 8, seed=22)):
+        a_bits = wl.hidden()
+        b_bits = workloads.RouterWorkload(wl.name, wl.T, wl.H, wl.E, wl.k, seed=wl.seed + 100).hidden()
+        w_bits = wl.gate_weight()
+        a, b = to_device_bf16(a_bits), to_device_bf16(b_bits)
+        w = to_device_bf16(w_bits)
+        x = torch.empty_like(a)
+        results = []
+        for src in (a, b, a, b):
+            x.copy_(src)  # the preceding kernel writes the gating's input
+            s, i = tk.fused_topk_gating(x, w, wl.k)
+            results.append((s.clone(), i.clone()))
+        torch.cuda.synchronize()
+        for bits, (s, i) in zip((a_bits, b_bits, a_bits, b_bits), results):
+            ref = oracle.fused_topk_gating(bits, w_bits, wl.k, want_logits=True)
+            parity.check(s.cpu().numpy(), i.cpu().numpy(), ref, label=wl.name)
