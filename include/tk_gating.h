@@ -206,8 +206,11 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
 
 /*
  * tk_gating_device_error -- read the device error word of the current device
- * (bits set by kernels whose bounded waits expired; 0 = none) into *word, and
- * clear it when `clear` is non-zero.  Synchronises the device.  Returns
+ * into *word (0 = none), and clear it when `clear` is non-zero.  Bits: 0..4 a
+ * bounded wait expired (producer, MMA, epilogue, drain, cluster); 5 an index
+ * check failed and its access was skipped (only in the checked build,
+ * libtk_gating_debug.so, compiled with TK_GATING_DEBUG); 8 an expert-parallel
+ * row address was not 16-byte aligned.  Synchronises the device.  Returns
  * TK_ERR_DEVICE_TIMEOUT when the word is non-zero, TK_OK otherwise.
  */
 TK_API tk_status tk_gating_device_error(uint32_t* word, int32_t clear);

@@ -9,7 +9,10 @@ import threading
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_PKG)
 HEADER = os.path.join(_ROOT, "include", "tk_gating.h")
-_LIB_PATH = os.path.join(_PKG, "libtk_gating.so")
+# TK_GATING_DEBUG=1 in the environment selects the build with the kernels' index
+# checks compiled in (python -m moe_router_gating_b200.build --debug)
+_LIB_PATH = os.path.join(_PKG, "libtk_gating_debug.so" if os.environ.get("TK_GATING_DEBUG", "0") not in ("", "0")
+                         else "libtk_gating.so")
 
 TK_OK = 0
 TK_ERR_INVALID_ARG = -1
@@ -51,7 +54,8 @@ def library() -> ctypes.CDLL:
         if _lib is None:
             if not os.path.exists(_LIB_PATH):
                 raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
-                                   "`python -m moe_router_gating_b200.build` (needs nvcc)")
+                                   "`python -m moe_router_gating_b200.build` (add --debug for the checked build; "
+                                   "needs nvcc)")
             lib = ctypes.CDLL(_LIB_PATH)
             vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
             lib.tk_gating_fused_topk.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp]

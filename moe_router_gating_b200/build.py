@@ -1,7 +1,8 @@
 """Build the in-tree CUDA library ``libtk_gating.so`` for sm_100a with nvcc.
 
-Usage: ``python -m moe_router_gating_b200.build [--verbose]`` (``--verbose``
-prints ptxas register / shared-memory usage).  Rebuilds only when a source or
+Usage: ``python -m moe_router_gating_b200.build [--verbose] [--debug]``
+(``--verbose`` prints ptxas register / shared-memory usage; ``--debug`` builds
+``libtk_gating_debug.so`` with the kernels' index checks compiled in).  Rebuilds only when a source or
 the public header is newer than the library.
 """
 from __future__ import annotations
@@ -19,6 +20,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtk_gating.so")
+# the same library with the kernels' index checks compiled in (TK_GATING_DEBUG)
+DEBUG_LIB = os.path.join(PKG, "libtk_gating_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -69,25 +72,30 @@ def gating_kernel_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB):
+def is_stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
     """Compile every csrc/*.cu to an object in parallel (the bf16 and FP8 kernel
-    instances live in separate translation units), then link the library."""
-    if not force and not is_stale():
-        return LIB
-    objdir = os.path.join(PKG, f"_build_{os.getpid()}")
+    instances live in separate translation units), then link the library.
+    ``debug`` builds libtk_gating_debug.so, with the kernels' index checks
+    (TK_GATING_DEBUG: a failed check sets a bit of the device error word and
+    skips the access)."""
+    target = DEBUG_LIB if debug else LIB
+    if not force and not is_stale(target):
+        return target
+    objdir = os.path.join(PKG, f"_build_{'debug_' if debug else ''}{os.getpid()}")
     os.makedirs(objdir, exist_ok=True)
     try:
         procs = []
         for src in sources():
             obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
-            cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+            cmd = [nvcc(), *NVCC_FLAGS, *(["-DTK_GATING_DEBUG"] if debug else []), "-I", INCLUDE, "-I", CSRC, "-c",
+                   src, "-o", obj]
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
             procs.append((src, obj, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
@@ -100,13 +108,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
                 failed.append(os.path.basename(src))
         if failed:
             raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(failed)})")
-        tmp = LIB + f".tmp{os.getpid()}"
+        tmp = target + f".tmp{os.getpid()}"
         subprocess.check_call([nvcc(), *LINK_FLAGS, *[obj for _, obj, _ in procs], "-o", tmp])
-        os.replace(tmp, LIB)
+        os.replace(tmp, target)
     finally:
         shutil.rmtree(objdir, ignore_errors=True)
-    return LIB
+    return target
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="--verbose" in sys.argv))
+    print(build(force=True, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

@@ -512,6 +512,9 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
         for (int c0 = 0; c0 < ncols; c0 += 64) {
           uint32_t r0[32], r1[32];
           const bool second = c0 + 32 < ncols;  // warp-uniform
+          // the columns read stay inside this CTA's tensor-memory allocation
+          if (!TK_CHECK(((chunk_addr - tmem_base) & 0xFFFFu) + c0 + (second ? 64u : 32u) <= p.tmem_cols, p.err_word))
+            break;
           tmem_ld_32(chunk_addr + c0, r0);
           if (second) tmem_ld_32(chunk_addr + c0 + 32, r1);
           tmem_ld_wait();
@@ -545,6 +548,8 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
         // its ring is idle: the upper lanes
         // hand their lists to the lower lanes of the same rows through it.
         const int m = (quad & 1) * 32 + lane;  // row within this CTA's 64
+        // the hand-over area (64 rows of KMAX floats, then of KMAX ids) lies inside the idle ring
+        if (!TK_CHECK(BLOCK_M * KMAX * 8 <= p.stages * KB_PER_STAGE * A_STAGE_BYTES, p.err_word)) break;
         float* xv = reinterpret_cast<float*>(sA) + m * KMAX;
         int32_t* xi = reinterpret_cast<int32_t*>(sA + BLOCK_M * KMAX * 4) + m * KMAX;
         if (upper) {

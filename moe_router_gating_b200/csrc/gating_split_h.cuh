@@ -280,10 +280,17 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
           const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
           const int t = quad * 32 + lane;  // tile-local row of this thread
           float* row = staging + static_cast<size_t>(t) * p.row_stride;
+          const int ring_bytes = p.stages * p.kps * (A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES);
           // 64 columns per tensor-memory round trip
           for (int c0 = 0; c0 < pass_cols; c0 += 64) {
             uint32_t v[2][32];
             const bool second = c0 + 32 < pass_cols;  // warp-uniform
+            // tensor-memory columns inside the allocation; staged row inside the idle ring
+            if (!TK_CHECK(col0 + c0 + (second ? 64 : 32) <= static_cast<int>(p.tmem_cols) &&
+                              (BLOCK_M - 1) * p.row_stride * 4 + (c0 + (second ? 64 : 32)) * 4 <= ring_bytes &&
+                              c0 + (second ? 64 : 32) <= p.row_stride,
+                          p.err_word))
+              break;
             tmem_ld_32(lane_base + c0, v[0]);
             if (second) tmem_ld_32(lane_base + c0 + 32, v[1]);
             tmem_ld_wait();
@@ -352,6 +359,8 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
         float* dump = p.logits == nullptr ? nullptr
                                           : p.logits + (static_cast<int64_t>(tile) * BLOCK_M + t_own) * p.E + ebase;
         for (int c = 4 * seg; c < pass_cols; c += 4 * group) {
+          // the pulled columns lie inside the staged row of every CTA
+          if (!TK_CHECK(c + 4 <= p.row_stride && t_own < BLOCK_M, p.err_word)) break;
           const float4 acc = column_quad(c);
           if (dump != nullptr) {
             dump[c] = acc.x;
@@ -374,10 +383,14 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
 
   // ---------------- merge the segments, softmax, store ----------------
   merge_lane_groups(top, group);
-  if (active && seg == 0) {
+  {
     const int t_local = static_cast<int>(r) + C * slot;
     const int64_t row = static_cast<int64_t>(tile) * BLOCK_M + t_local;
-    top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+    if (group >= p.k) {  // every lane of the group holds the list: one entry per lane
+      group_softmax_store(top, p.k, group, active, p.scores + row * p.k, p.ids + row * p.k);
+    } else if (active && seg == 0) {
+      top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+    }
   }
   if (clock_cta) record_launch_clock(p.clock, t0_ns, t0_clk);
 }

@@ -10,6 +10,10 @@
 #include "tk_gating.h"
 #include "route.cuh"
 
+namespace tkg {
+uint32_t* device_error_word();  // tk_gating.cu: the device error word of the current device
+}
+
 namespace {
 
 int64_t round_up64(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
@@ -143,6 +147,8 @@ tk_status launch_route(const tk_route_plan& pl, const int32_t* ids, int64_t n, i
   p.offsets = offsets;
   p.sorted_slots = sorted_slots;
   p.slot_pos = slot_pos;
+  p.err_word = tkg::device_error_word();
+  if (p.err_word == nullptr) return TK_ERR_CUDA;
 
   if (pl.ctas > 1) {
     cudaLaunchConfig_t cfg = {};

@@ -29,6 +29,8 @@
 
 #include <cstdint>
 
+#include "sm100_ptx.cuh"
+
 namespace tkg {
 
 constexpr int ROUTE_WARPS = 32;
@@ -48,6 +50,7 @@ struct RouteParams {
   int32_t* offsets;      // [E + 1]
   int32_t* sorted_slots; // [n]
   int32_t* slot_pos;     // [n]
+  uint32_t* err_word;    // device error word (debug-build index checks)
 };
 
 __device__ __forceinline__ uint32_t route_lanemask_lt() {
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
       // the lowest lane of each group moves its expert's position past the group
       if (e[i] >= 0 && (grp & lt) == 0) my[e[i]] += __popc(grp);
       __syncwarp();
-      if (s < end) {
+      if (s < end && TK_CHECK(pos < p.n, p.err_word)) {
         p.slot_pos[s] = pos;
         if (pos >= 0) p.sorted_slots[pos] = static_cast<int32_t>(s);
       }

@@ -28,7 +28,19 @@ enum : uint32_t {
   ERR_WAIT_EPILOGUE = 1u << 2,
   ERR_WAIT_DRAIN = 1u << 3,
   ERR_WAIT_CLUSTER = 1u << 4,
+  ERR_BOUNDS = 1u << 5,  // debug builds: an index check failed; the access was skipped
 };
+
+// Debug builds (compiled with -DTK_GATING_DEBUG, libtk_gating_debug.so): TK_CHECK
+// records ERR_BOUNDS in the device error word and yields false when `cond` does
+// not hold, so the guarded access is skipped; in release builds it is `true` and
+// costs nothing.  It guards indexes that hold by construction -- the stand-in
+// for a memory checker, which this pool does not offer.
+#ifdef TK_GATING_DEBUG
+#define TK_CHECK(cond, err_word) ((cond) ? true : (atomicOr((err_word), ::tkg::ERR_BOUNDS), false))
+#else
+#define TK_CHECK(cond, err_word) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

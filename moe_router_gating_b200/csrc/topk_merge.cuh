@@ -66,3 +66,39 @@ __device__ __forceinline__ void merge_lane_groups(RowTopK<L>& t, int group) {
 }
 
 }  // namespace tkg
+
+namespace tkg {
+
+// softmax_store by a group of >= k lanes that all hold the same sorted list:
+// lane j (j < k, j = the lane's position in its group) computes exp(v_j - v_0),
+// every lane gathers the k terms by shuffles and sums them in the order
+// j = 0 .. k-1, and lane j stores entry j -- the arithmetic of
+// RowTopK::softmax_store, spread over the lanes.  `store` is false for lanes
+// whose group has no row to write (they still take part in the shuffles).
+// Every lane of the warp must call this with the same `group` (>= k).
+template <int L>
+__device__ __forceinline__ void group_softmax_store(const RowTopK<L>& t, int k, int group, bool store,
+                                                    float* __restrict__ score_row, int32_t* __restrict__ id_row) {
+  const int lane = static_cast<int>(threadIdx.x & 31);
+  const int j = lane & (group - 1);
+  const int base = lane - j;
+  float vj = t.v[0];
+  int32_t ij = t.i[0];
+#pragma unroll
+  for (int q = 1; q < L; ++q) {
+    vj = q == j ? t.v[q] : vj;
+    ij = q == j ? t.i[q] : ij;
+  }
+  const float ex = j < k ? expf(vj - t.v[0]) : 0.0f;
+  float sum = 0.0f;
+  for (int q = 0; q < L; ++q) {  // the same order as softmax_store
+    const float e = __shfl_sync(0xffffffffu, ex, base + (q < group ? q : 0));
+    sum += q < k ? e : 0.0f;
+  }
+  if (store && j < k) {
+    score_row[j] = ex / sum;
+    id_row[j] = ij;
+  }
+}
+
+}  // namespace tkg

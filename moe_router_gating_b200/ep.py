@@ -18,7 +18,7 @@ per-expert counts, gathered over the process group, and, once per group,
 the inter-process handles of every rank's buffers.
 
 With one rank everything stays on the caller's stream, except one read of the
-received row count (the length of the returned view).  With several, ranks
+routing offsets (to size the returned view and check every rank's capacity).  With several, ranks
 order their steps with process-group barriers after synchronising their
 stream (each rank's dispatch must be complete before any expert reads a
 receive buffer, and every expert output before any combine reads it).
@@ -65,6 +65,31 @@ class ExchangePlan:
     recv_rows: list          # rows each rank receives
     recv_offsets: list       # per rank q: its experts' first rows in its buffer (length E/R + 1)
     dest_row: list           # for `rank` as source: the first row of its block of expert e
+
+
+def received_rows(offsets_all, R: int, E: int) -> list:
+    """Rows each rank receives, from every rank's routing offsets ([R][E + 1])."""
+    per = E // R
+    rows = [0] * R
+    for s in range(R):
+        o = offsets_all[s]
+        for q in range(R):
+            rows[q] += int(o[(q + 1) * per]) - int(o[q * per])
+    return rows
+
+
+def check_capacities(offsets_all, capacities) -> list:
+    """The rows each rank receives; ValueError when one exceeds its capacity.
+    Every rank runs this on the same gathered offsets, so all of them refuse
+    together and no rank writes past another's buffer."""
+    R = len(capacities)
+    E = len(offsets_all[0]) - 1
+    rows = received_rows(offsets_all, R, E)
+    over = [q for q in range(R) if rows[q] > capacities[q]]
+    if over:
+        q = over[0]
+        raise ValueError(f"rank {q} would receive {rows[q]} rows; its capacity is {capacities[q]}")
+    return rows
 
 
 def exchange_plan(counts, rank: int) -> ExchangePlan:
@@ -212,13 +237,15 @@ class ExpertParallelGroup:
         if self.R == 1:
             bases = [self.recv.data_ptr()]
             out_bases = [self.output.data_ptr()]
+            self.capacities = [self.capacity]
         else:
-            mine = (ipc_handle(self.recv), ipc_handle(self.output))
+            mine = (ipc_handle(self.recv), ipc_handle(self.output), self.capacity)
             allh = [None] * self.R
             dist.all_gather_object(allh, mine, group=group)
             bases, out_bases = [], []
+            self.capacities = [int(c) for (_, _, c) in allh]
             with torch.cuda.device(self.device):
-                for q, (hr, ho) in enumerate(allh):
+                for q, (hr, ho, _) in enumerate(allh):
                     if q == self.rank:
                         bases.append(self.recv.data_ptr())
                         out_bases.append(self.output.data_ptr())
@@ -269,10 +296,10 @@ class ExpertParallelGroup:
             raise ValueError(f"tokens must be bf16 [T, {self.H}]")
         offsets, sorted_slots, slot_pos = b.route(expert_ids, self.E, stream=stream)
         offsets_all = self._gather_offsets(offsets)
+        # every rank checks every destination (the same numbers on all ranks): the
+        # dispatch below writes into other ranks' buffers
+        recv_rows = check_capacities(offsets_all.cpu().tolist(), self.capacities)[self.rank]
         rows, out_rows, recv_offsets = rows_table(offsets_all, self.rank, self.bases, self.out_bases, self.H, stream)
-        recv_rows = int(recv_offsets[-1])  # the receive view's length (waits for the table)
-        if recv_rows > self.capacity:
-            raise ValueError(f"rank {self.rank} would receive {recv_rows} rows; capacity is {self.capacity}")
         self._barrier(stream)  # every receive buffer is free
         dispatch_rows(tokens, expert_ids, offsets, sorted_slots, rows, self.E, stream)
         self._barrier(stream)  # every rank's rows have landed

@@ -116,3 +116,15 @@ def test_two_gloo_ranks_exchange_offsets_and_place_rows():
     want = ep_oracle.dispatch(toks, ids, E)
     for r in range(world):
         assert np.array_equal(got[r], want.rows[r]), r
+
+
+def test_capacity_check_sees_every_destination():
+    # two ranks, four experts: rank 0 holds experts 0-1, rank 1 experts 2-3
+    offsets_all = [[0, 3, 5, 9, 10],    # rank 0's routing: counts 3, 2, 4, 1
+                   [0, 1, 1, 6, 8]]     # rank 1's routing: counts 1, 0, 5, 2
+    assert ep.received_rows(offsets_all, 2, 4) == [3 + 2 + 1 + 0, 4 + 1 + 5 + 2]
+    assert ep.check_capacities(offsets_all, [6, 12]) == [6, 12]
+    with pytest.raises(ValueError, match="rank 1"):
+        ep.check_capacities(offsets_all, [100, 11])   # another rank's buffer would overflow
+    with pytest.raises(ValueError, match="rank 0"):
+        ep.check_capacities(offsets_all, [5, 100])
