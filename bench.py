@@ -80,6 +80,11 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback (earlier measurement on this pool)"
 
 
+def of_peaks(peak_src: str) -> str:
+    """How a roofline fraction names its denominator: measured on this machine, or the fallback."""
+    return "of measured" if peak_src.startswith("measured") else "of fallback"
+
+
 def workload_desc(wl):
     extra = ""
     if wl.kind == "skew":
@@ -487,8 +492,8 @@ def roofline_of(wl, launch_ms: float, fp8: bool, peaks: dict, peak_src: str) -> 
     primary, secondary = (hbm, tc) if t_hbm >= t_tc_burst else (tc, hbm)
     roof = dict(primary)
     roof.update({
-        "peak_source": (f"{peak_src}; HBM = copy GB/s (of measured); tensor = cuBLAS bf16 burst TFLOP/s "
-                        f"(of measured){'; x2 for FP8 (nominal FP8/bf16 ratio)' if fp8 else ''}"),
+        "peak_source": (f"{peak_src}; HBM = copy GB/s ({of_peaks(peak_src)}); tensor = cuBLAS bf16 burst "
+                        f"TFLOP/s ({of_peaks(peak_src)}){'; x2 for FP8 (nominal FP8/bf16 ratio)' if fp8 else ''}"),
         "roofline_frac": max(t_hbm, t_tc_burst) / t_s,
         "roofline_frac_sustained": max(t_hbm, t_tc_sust) / t_s,
         "tensor_frac_sustained": tc_ach / tc_sust,
@@ -780,7 +785,7 @@ def run_route_ours(args, wl):
         ach = bytes_alg / (ms_per_step / 1e3) / 1e9
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": ach / peaks["hbm_gbs"], "traffic": None,
-                            "peak_source": f"{peak_src}; copy GB/s (of measured)",
+                            "peak_source": f"{peak_src}; copy GB/s ({of_peaks(peak_src)})",
                             "algorithmic_bytes_per_step": bytes_alg,
                             "note": "two launches per step (count, then scatter); time of the pair"}
         line["e2e"] = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 4 * T * k,
@@ -864,7 +869,7 @@ def run_ep_ours(args, wl):
                      "dispatch_gbs": d_bytes / (t_d / 1e3) / 1e9, "combine_gbs": c_bytes / (t_c / 1e3) / 1e9,
                      "dispatch_frac": d_bytes / (t_d / 1e3) / 1e9 / peaks["hbm_gbs"],
                      "combine_frac": c_bytes / (t_c / 1e3) / 1e9 / peaks["hbm_gbs"],
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": f"{peak_src}; copy GB/s",
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": f"{peak_src}; copy GB/s ({of_peaks(peak_src)})",
                      "algorithmic_bytes": {"dispatch": d_bytes, "combine": c_bytes}},
         "gpu_launches": args.steps * 2,
         "clocks": sampler.summary(),
