@@ -10,7 +10,8 @@ router, T=65536 tokens, H=7168, E=256 experts, k=8 (hidden 940 MB > L2).
 ``--precision fp8`` times the FP8 (E4M3) entry point on the workload's inputs
 quantized per token (hidden) and per expert (gate).  ``--op route`` times the routing metadata (per-expert offsets, the expert-grouped
 order and each assignment's position) of seeded ids of the workload's T x k
-shape; ``--op gating_route`` times gating followed by routing of its ids.
+shape; ``--op gating_route`` times gating and the routing of its ids in one call (the counts per expert
+taken by the gating kernel), beside the gating alone and the two separate calls.
 
 Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one process per GPU)
 every rank gates its own batch of T tokens (token shards, no collective on the
@@ -154,7 +155,7 @@ def run_reference(args, wl):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    def __init__(self, local_rank: int, period_s: float = 0.001):
+    def __init__(self, local_rank: int, period_s: float = 0.0005):
         self.samples = []
         self.period = period_s
         self._stop = threading.Event()
@@ -181,16 +182,21 @@ class ClockSampler:
             self.error = repr(e)
 
     def _run(self):
+        # only the SM clock and the event reasons every period (cheap queries);
+        # the power reading is slower and is taken every 8th sample
         p, h = self._nvml, self._h
+        power = None
+        i = 0
         while not self._stop.is_set():
             try:
                 sm = p.nvmlDeviceGetClockInfo(h, p.NVML_CLOCK_SM)
-                util = p.nvmlDeviceGetUtilizationRates(h).gpu
                 reasons = self._reasons(h)
-                power = p.nvmlDeviceGetPowerUsage(h) / 1000.0
-                self.samples.append((sm, util, reasons, power))
+                if i % 8 == 0:
+                    power = p.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((sm, reasons, power))
             except Exception as e:
                 self.error = repr(e)
+            i += 1
             self._stop.wait(self.period)
 
     def __enter__(self):
@@ -212,7 +218,7 @@ class ClockSampler:
         reasons = set()
         for s in self.samples:
             for bit, name in NVML_REASONS.items():
-                if s[2] & bit and name != "gpu_idle":
+                if s[1] & bit and name != "gpu_idle":
                     reasons.add(name)
         return {
             "sm_mhz": statistics.median([s[0] for s in self.samples]) if self.samples else None,
@@ -220,8 +226,8 @@ class ClockSampler:
             "sm_max_mhz": self.max_mhz,
             "reasons": sorted(reasons),
             "samples": len(self.samples),
-            "power_w_max": max([s[3] for s in self.samples]) if self.samples else None,
-            "source": "NVML (same counters as nvidia-smi), sampled every %.0f ms during the timed region"
+            "power_w_max": max([s[2] for s in self.samples if s[2] is not None], default=None),
+            "source": "NVML (same counters as nvidia-smi), sampled every %.1f ms during the timed region"
                       % (self.period * 1e3),
         }
 
@@ -701,10 +707,22 @@ def run_route_ours(args, wl):
         scores = torch.empty((T, k), dtype=torch.float32, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
-    def step():
-        if chain:
-            tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream)
-        tk.route(ids, E, offsets, sorted_slots, slot_pos, stream=stream)
+    if chain:
+        # gating and routing in one call: the gating kernel counts the assignments
+        # per expert, the placing kernel follows (tk_gating_fused_topk_route)
+        ws = tk.route_workspace(T, k, E, dev)
+        H = x.shape[1]
+
+        def step():
+            st = tk.fused_topk_gating_route_ptr(x.data_ptr(), w.data_ptr(), T, H, E, k, scores.data_ptr(),
+                                                ids.data_ptr(), offsets.data_ptr(), sorted_slots.data_ptr(),
+                                                slot_pos.data_ptr(), ws.data_ptr(), ws.numel() * 4,
+                                                stream.cuda_stream)
+            if st != tk.TK_OK:
+                raise SystemExit(f"tk_gating_fused_topk_route: {tk.status_string(st)}")
+    else:
+        def step():
+            tk.route(ids, E, offsets, sorted_slots, slot_pos, stream=stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -725,18 +743,25 @@ def run_route_ours(args, wl):
     elapsed_ms = sum(per)
     ms_per_step = elapsed_ms / args.steps
     value = T * args.steps / (elapsed_ms / 1e3)
-    gating_alone_ms = None
+    gating_alone_ms = chained_ms = None
     if chain:
-        # the gating call alone, timed the same way in the same run: the routing's added cost
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for a, b in evs:
-            flush.zero_()
-            a.record(stream)
-            tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream)
-            b.record(stream)
-        torch.cuda.synchronize(dev)
-        gating_alone_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+        # timed the same way in the same run: the gating call alone (the routing's
+        # added cost), and the two separate calls (gating, then tk_gating_route,
+        # which counts the ids in a launch of its own)
+        def timed(fn):
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize(dev)
+            return sum(a.elapsed_time(b) for a, b in evs) / args.steps
+
+        gating_alone_ms = timed(lambda: tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream))
+        chained_ms = timed(lambda: (tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream),
+                                    tk.route(ids, E, offsets, sorted_slots, slot_pos, stream=stream)))
 
     # end to end: pinned host ids -> device, route, the three outputs -> pinned host
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
@@ -775,12 +800,15 @@ def run_route_ours(args, wl):
                    "T": T, "k": k, "E": E,
                    "l2": "L2 flushed (256 MB write) before every timed step; each step timed alone",
                    "launch": plan},
-        "gpu_launches": args.steps * (3 if chain else 2),
+        "gpu_launches": args.steps * 2,  # gating + placing kernel, or counting + placing kernel
         "clocks": sampler.summary(),
     }
     if chain:
+        line["path"] = "tk_gating_fused_topk_route (counts taken in the gating epilogue)"
         line["gating_alone_ms_per_step"] = gating_alone_ms
         line["routing_added_us"] = (ms_per_step - gating_alone_ms) * 1e3
+        line["separate_calls_ms_per_step"] = chained_ms
+        line["separate_calls_routing_added_us"] = (chained_ms - gating_alone_ms) * 1e3
     if not chain:
         ach = bytes_alg / (ms_per_step / 1e3) / 1e9
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -24,6 +24,7 @@
  *     device; the caller allocates and owns every buffer.  The library keeps no
  *     per-call state.  Only tk_gating_route allocates device memory: a
  *     stream-ordered workspace that it frees on the same stream.
+ *     tk_gating_fused_topk_route uses a workspace that the caller owns.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls are asynchronous: they return once the work is enqueued.  Launch
  *     failures return TK_ERR_CUDA; faults inside a kernel surface at the
@@ -209,7 +210,9 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
  * into *word (0 = none), and clear it when `clear` is non-zero.  Bits: 0..4 a
  * bounded wait expired (producer, MMA, epilogue, drain, cluster); 5 an index
  * check failed and its access was skipped (only in the checked build,
- * libtk_gating_debug.so, compiled with TK_GATING_DEBUG); 8 an expert-parallel
+ * libtk_gating_debug.so, compiled with TK_GATING_DEBUG); 6 the routing counts
+ * taken by the gating disagreed with the ids (tk_gating_fused_topk_route
+ * given a workspace that was not zero); 8 an expert-parallel
  * row address was not 16-byte aligned.  Synchronises the device.  Returns
  * TK_ERR_DEVICE_TIMEOUT when the word is non-zero, TK_OK otherwise.
  */
@@ -273,6 +276,8 @@ typedef struct {
   int64_t workspace_bytes;    /* device workspace: ctas x round_up(E, 4) int32 counts, 0 when ctas == 1 */
   int32_t count_smem_bytes;   /* dynamic shared memory of the counting kernel */
   int32_t scatter_smem_bytes; /* dynamic shared memory of the placing kernel */
+  int64_t fused_workspace_bytes; /* workspace of tk_gating_fused_topk_route: the counts table and a
+                                    16-byte arrival counter (workspace_bytes + 16), 0 when ctas == 1 */
 } tk_route_plan;
 
 /*
@@ -312,6 +317,54 @@ TK_API tk_status tk_gating_route(const int32_t* ids, int64_t T, int32_t k, int32
  * tk_gating_route.  Makes no CUDA call.
  */
 TK_API tk_status tk_gating_route_plan(int64_t T, int32_t k, int32_t E, int32_t num_sms, tk_route_plan* plan);
+
+/*
+ * tk_gating_fused_topk_route -- tk_gating_fused_topk followed by
+ * tk_gating_route of its ids, with the routing's counting step done by the
+ * gating kernel: each selected (token, expert) assignment is added to a small
+ * table of per-expert counts (atomic adds in global memory) as the gating
+ * stores it (chenxutan.com, "TileKernels 深度解析", section 4.2 "MoE Routing":
+ * the counts per expert that dispatch starts from, taken where the ids are
+ * produced).  The placing kernel then reads the table instead of counting the
+ * ids in a launch of its own.  Outputs, layouts and results are exactly those
+ * of the two calls made one after the other.
+ *
+ *   hidden, gate_weight, T, H, E, k, scores, ids   as tk_gating_fused_topk.
+ *   offsets, sorted_slots, slot_pos                as tk_gating_route
+ *                                                  (4-byte aligned).
+ *   workspace     device, at least tk_route_plan.fused_workspace_bytes
+ *                 (tk_gating_route_plan of (T, k, E) on this device's SM
+ *                 count), 16-byte aligned; may be NULL when that is 0.  It
+ *                 must hold zeros when a call starts: zero it once after
+ *                 allocating it; every call leaves the part it used zero
+ *                 again, so one workspace serves any sequence of calls
+ *                 issued in order (one stream).  Calls that overlap need
+ *                 workspaces of their own.
+ *   workspace_bytes  its size.
+ *   stream        cudaStream_t (void*), may be NULL.
+ *
+ * Launches on `stream`: the gating kernel, then (up to 4096 assignments) the
+ * routing's one-CTA kernel -- the table is then not used -- or the placing
+ * kernel, launched as a programmatic dependent of the gating.  Allocates
+ * nothing.
+ *
+ * The placing kernel checks the table against the ids it reads: a CTA whose
+ * row of the table differs from its own count of its assignments (a workspace
+ * that was not zero) sets bit 6 of the device error word
+ * (tk_gating_device_error), and no position outside [0, T*k) is written; the
+ * routing outputs of that call are then not valid.  Zero the workspace again
+ * after bit 6 was reported (stale counts alone are cleared by the call itself,
+ * a stale arrival counter in the last 16 bytes is not).
+ *
+ * Errors: those of tk_gating_fused_topk and of tk_gating_route, and
+ *   TK_ERR_INVALID_ARG   workspace NULL or smaller than
+ *                        tk_route_plan.fused_workspace_bytes while that is > 0;
+ *   TK_ERR_ALIGNMENT     workspace not 16-byte aligned.
+ */
+TK_API tk_status tk_gating_fused_topk_route(const void* hidden, const void* gate_weight, int64_t T, int64_t H,
+                                            int64_t E, int32_t k, float* scores, int32_t* ids, int32_t* offsets,
+                                            int32_t* sorted_slots, int32_t* slot_pos, void* workspace,
+                                            int64_t workspace_bytes, void* stream);
 
 /*
  * tk_gating_route_static -- tk_gating_route without any allocation.

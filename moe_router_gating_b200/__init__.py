@@ -28,19 +28,23 @@ from ._binding import (  # noqa: F401
     fused_topk_gating_fp8_ptr,
     fused_topk_gating_host,
     fused_topk_gating_ptr,
+    fused_topk_gating_route,
+    fused_topk_gating_route_ptr,
     library,
     library_path,
     make_plan,
     route,
     route_plan,
     route_ptr,
+    route_workspace,
     route_static_ptr,
     set_wait_timeout_ns,
     status_string,
 )
 
 __all__ = [
-    "fused_topk_gating", "fused_topk_gating_fp8", "fused_topk_gating_host", "fused_topk_gating_ptr", "make_plan", "route", "route_plan",
+    "fused_topk_gating", "fused_topk_gating_fp8", "fused_topk_gating_host", "fused_topk_gating_ptr",
+    "fused_topk_gating_route", "fused_topk_gating_route_ptr", "route_workspace", "make_plan", "route", "route_plan",
     "route_ptr", "route_static_ptr", "device_error", "clock_counters",
     "set_wait_timeout_ns", "status_string", "TkGatingError", "library", "library_path",
 ]

@@ -40,7 +40,7 @@ class _Plan(ctypes.Structure):
 class _RoutePlan(ctypes.Structure):
     _fields_ = [("ctas", ctypes.c_int32), ("threads", ctypes.c_int32), ("warp_slots", ctypes.c_int64),
                 ("workspace_bytes", ctypes.c_int64), ("count_smem_bytes", ctypes.c_int32),
-                ("scatter_smem_bytes", ctypes.c_int32)]
+                ("scatter_smem_bytes", ctypes.c_int32), ("fused_workspace_bytes", ctypes.c_int64)]
 
 
 def library_path() -> str:
@@ -64,6 +64,8 @@ def library() -> ctypes.CDLL:
             lib.tk_gating_fused_topk_host.restype = ctypes.c_int
             lib.tk_gating_fused_topk_fp8.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp]
             lib.tk_gating_fused_topk_fp8.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_route.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, i64, vp]
+            lib.tk_gating_fused_topk_route.restype = ctypes.c_int
             lib.tk_gating_fused_topk_logits.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
             lib.tk_gating_fused_topk_logits.restype = ctypes.c_int
             lib.tk_gating_fused_topk_fp8_logits.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
@@ -158,6 +160,78 @@ def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, st
             st = fn(*args, _stream_handle(stream, hidden.device))
     _check(st, name)
     return scores, ids
+
+
+_route_ws_lock = threading.Lock()
+_route_ws = {}  # (device index, stream handle) -> zeroed int32 workspace of fused_topk_gating_route
+
+
+def route_workspace(T: int, k: int, E: int, device=None):
+    """A zeroed int32 CUDA tensor large enough to serve as the workspace of
+    ``fused_topk_gating_route`` for (T, k, E) on ``device`` (at least 4 elements).
+    Zero it again only if a call reported bit 6 of the device error word."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    nbytes = route_plan(T, k, E, sms)["fused_workspace_bytes"]
+    return torch.zeros(max(4, (nbytes + 3) // 4), dtype=torch.int32, device=dev)
+
+
+def fused_topk_gating_route_ptr(hidden: int, gate_weight: int, T: int, H: int, E: int, k: int, scores: int, ids: int,
+                                offsets: int, sorted_slots: int, slot_pos: int, workspace: int, workspace_bytes: int,
+                                stream: int = 0) -> int:
+    """Raw C-ABI call of the fused gating + routing entry point (integer device
+    pointers); returns the tk_status."""
+    return int(library().tk_gating_fused_topk_route(hidden, gate_weight, T, H, E, k, scores, ids, offsets,
+                                                    sorted_slots, slot_pos, workspace, workspace_bytes, stream))
+
+
+def fused_topk_gating_route(hidden, gate_weight, top_k: int, workspace=None, stream=None):
+    """Gating and the routing metadata of its ids in one call, the counts per
+    expert taken by the gating kernel: ``(scores, ids, offsets, sorted_slots,
+    slot_pos)``, the results of ``fused_topk_gating`` and then ``route``.
+
+    ``workspace`` (int32 CUDA tensor, zero before its first use, left zero by
+    every call) defaults to one the binding keeps per device and stream; pass
+    one of ``route_workspace``'s when capturing the call into a CUDA graph."""
+    import torch
+    if hidden.dtype != torch.bfloat16 or gate_weight.dtype != torch.bfloat16:
+        raise TypeError("hidden and gate_weight must be torch.bfloat16")
+    if hidden.dim() != 2 or gate_weight.dim() != 2 or hidden.shape[1] != gate_weight.shape[0]:
+        raise ValueError(f"shapes {tuple(hidden.shape)} @ {tuple(gate_weight.shape)} do not chain")
+    if not hidden.is_cuda or hidden.device != gate_weight.device or not hidden.is_contiguous() \
+            or not gate_weight.is_contiguous():
+        raise ValueError("hidden and gate_weight must be contiguous CUDA tensors on one device")
+    T, H = hidden.shape
+    E = gate_weight.shape[1]
+    k = int(top_k)
+    dev = hidden.device
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        if workspace is None:
+            key = (dev.index, int(s.cuda_stream))
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            need = route_plan(T, k, E, sms)["fused_workspace_bytes"]
+            with _route_ws_lock:
+                workspace = _route_ws.get(key)
+                if workspace is None or workspace.numel() * 4 < need:
+                    with torch.cuda.stream(s):  # zeroed in the order of the calls that use it
+                        workspace = torch.zeros(max(4, (need + 3) // 4), dtype=torch.int32, device=dev)
+                    _route_ws[key] = workspace
+        if workspace.dtype != torch.int32 or not workspace.is_cuda or workspace.device != dev \
+                or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous int32 CUDA tensor on the inputs' device")
+        scores = torch.empty((T, k), dtype=torch.float32, device=dev)
+        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        sorted_slots = torch.empty(T * k, dtype=torch.int32, device=dev)
+        slot_pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+        st = library().tk_gating_fused_topk_route(
+            hidden.data_ptr(), gate_weight.data_ptr(), T, H, E, k, scores.data_ptr(), ids.data_ptr(),
+            offsets.data_ptr(), sorted_slots.data_ptr(), slot_pos.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * 4, int(s.cuda_stream))
+    _check(st, "tk_gating_fused_topk_route")
+    return scores, ids, offsets, sorted_slots, slot_pos
 
 
 def _check_logits(logits, T: int, E: int, device) -> None:

@@ -28,6 +28,7 @@ struct LaunchEnv {
   uint32_t* err_word;     // device error word of the bounded waits
   uint64_t timeout_ns;    // bounded-wait limit
   uint64_t* clock;        // SM-clock counters of the launches (cycles, ns, launches)
+  RouteCounts route;      // per-expert counts of the stored ids by routing range; table null: none
 };
 
 // Shared-memory limits (and non-portable cluster sizes) of every kernel instance

@@ -133,6 +133,7 @@ tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const C
     sp.gscale = gscale;
     sp.logits = logits;
     sp.clock = env.clock;
+    sp.route = env.route;
     const int mc = env.max_split_cluster;
     // lists of 4 also serve k = 1, 2 (fewer kernel instances to build; an
     // insertion into 4 slots costs little more than into 1 or 2)
@@ -166,6 +167,7 @@ tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const C
   prm.gscale = gscale;
   prm.logits = logits;
   prm.clock = env.clock;
+  prm.route = env.route;
 
   if (k <= 4) return launch_row_variant<4, FP8>(pl, mx, mx64, mw, prm, stream);
   if (k <= 8) return launch_row_variant<8, FP8>(pl, mx, mx64, mw, prm, stream);

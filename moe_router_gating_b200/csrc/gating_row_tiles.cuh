@@ -57,6 +57,7 @@
 
 #include "sm100_ptx.cuh"
 #include "topk_epilogue.cuh"
+#include "route_counts.cuh"
 #include "topk_merge.cuh"
 
 namespace tkg {
@@ -93,6 +94,7 @@ struct RowTileParams {
   const float* gscale;  // FP8 only: per-expert scales [E]
   float* logits;        // optional [T, E]: every logit the selection ranks is also stored (verification)
   uint64_t* clock;      // SM-clock counters: the first CTA adds its cycles and ns (and 1) per launch
+  RouteCounts route;    // optional per-expert counts of the stored ids by routing range (route_counts.cuh)
 };
 
 // K elements of H per K slice: one 128-byte swizzle row of bf16 or of FP8 values.
@@ -542,7 +544,10 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
       if (w.eg + 1 < EG) continue;  // the tile's next expert group follows
       if (!w.half) {
         const int64_t row = static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
-        if (row < p.T) top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+        if (row < p.T) {
+          top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+          if (p.route.table != nullptr) route_count_row(p.route, top, p.k, row, p.E);
+        }
       } else {
         // A half tile is a CTA's last tile (and this its last expert group), so
         // its ring is idle: the upper lanes
@@ -570,7 +575,10 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           }
           merge_sorted(top, bv, bi);
           const int64_t row = static_cast<int64_t>(w.row0) + rank * (BLOCK_M / 2) + m;
-          if (row < p.T) top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+          if (row < p.T) {
+            top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+            if (p.route.table != nullptr) route_count_row(p.route, top, p.k, row, p.E);
+          }
         }
       }
     }

@@ -44,6 +44,7 @@
 #include "gating_row_tiles.cuh"
 #include "sm100_ptx.cuh"
 #include "topk_epilogue.cuh"
+#include "route_counts.cuh"
 #include "topk_merge.cuh"
 
 namespace tkg {
@@ -73,6 +74,7 @@ struct SplitHParams {
   const float* gscale;  // FP8 only: per-expert scales [E]
   float* logits;        // optional [T, E]: every logit the selection ranks is also stored (verification)
   uint64_t* clock;      // SM-clock counters: the first CTA adds its cycles and ns (and 1) per launch
+  RouteCounts route;    // optional per-expert counts of the stored ids by routing range (route_counts.cuh)
 };
 
 template <int KMAX, int C, bool FP8>
@@ -280,7 +282,7 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
           const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col0);
           const int t = quad * 32 + lane;  // tile-local row of this thread
           float* row = staging + static_cast<size_t>(t) * p.row_stride;
-          const int ring_bytes = p.stages * p.kps * (A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES);
+          [[maybe_unused]] const int ring_bytes = p.stages * p.kps * (A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES);
           // 64 columns per tensor-memory round trip
           for (int c0 = 0; c0 < pass_cols; c0 += 64) {
             uint32_t v[2][32];
@@ -388,8 +390,10 @@ __global__ void __launch_bounds__(SPLIT_THREADS, 1)
     const int64_t row = static_cast<int64_t>(tile) * BLOCK_M + t_local;
     if (group >= p.k) {  // every lane of the group holds the list: one entry per lane
       group_softmax_store(top, p.k, group, active, p.scores + row * p.k, p.ids + row * p.k);
+      if (p.route.table != nullptr) group_route_count(p.route, top, p.k, group, active, row, p.E);
     } else if (active && seg == 0) {
       top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+      if (p.route.table != nullptr) route_count_row(p.route, top, p.k, row, p.E);
     }
   }
   if (clock_cta) record_launch_clock(p.clock, t0_ns, t0_clk);

@@ -52,6 +52,9 @@ tk_status route_plan_impl(int64_t T, int32_t k, int32_t E, int32_t num_sms, tk_r
   plan->threads = tkg::ROUTE_THREADS;
   plan->warp_slots = L;
   plan->workspace_bytes = G > 1 ? G * round_up64(E, 4) * 4 : 0;  // one CTA needs no table
+  // counts from the gating: the table, then the scatter CTAs' arrival counter
+  // (16 bytes keep the size a multiple of 16)
+  plan->fused_workspace_bytes = G > 1 ? plan->workspace_bytes + 16 : 0;
   plan->count_smem_bytes = count_smem_bytes(E);
   plan->scatter_smem_bytes = scatter_smem_bytes(E);
   return TK_OK;
@@ -74,6 +77,13 @@ bool set_route_smem(Kernel kernel, int32_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
+template <int NB>
+bool set_scatter_smem(int32_t bytes) {
+  return set_route_smem(tkg::route_scatter_kernel<NB, tkg::ROUTE_ONE_CTA>, bytes) &&
+         set_route_smem(tkg::route_scatter_kernel<NB, tkg::ROUTE_TABLE>, bytes) &&
+         set_route_smem(tkg::route_scatter_kernel<NB, tkg::ROUTE_FUSED>, bytes);
+}
+
 const RouteDevice* route_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -93,14 +103,9 @@ const RouteDevice* route_device() {
     return &d;
   }
   if (!set_route_smem(tkg::route_count_kernel, count_smem_bytes(TK_ROUTE_MAX_EXPERTS)) ||
-      !set_route_smem(tkg::route_scatter_kernel<4, true>, scatter_smem_bytes(16)) ||
-      !set_route_smem(tkg::route_scatter_kernel<4, false>, scatter_smem_bytes(16)) ||
-      !set_route_smem(tkg::route_scatter_kernel<6, true>, scatter_smem_bytes(64)) ||
-      !set_route_smem(tkg::route_scatter_kernel<6, false>, scatter_smem_bytes(64)) ||
-      !set_route_smem(tkg::route_scatter_kernel<8, true>, scatter_smem_bytes(256)) ||
-      !set_route_smem(tkg::route_scatter_kernel<8, false>, scatter_smem_bytes(256)) ||
-      !set_route_smem(tkg::route_scatter_kernel<10, true>, scatter_smem_bytes(TK_ROUTE_MAX_EXPERTS)) ||
-      !set_route_smem(tkg::route_scatter_kernel<10, false>, scatter_smem_bytes(TK_ROUTE_MAX_EXPERTS))) {
+      !set_scatter_smem<4>(scatter_smem_bytes(16)) || !set_scatter_smem<6>(scatter_smem_bytes(64)) ||
+      !set_scatter_smem<8>(scatter_smem_bytes(256)) ||
+      !set_scatter_smem<10>(scatter_smem_bytes(TK_ROUTE_MAX_EXPERTS))) {
     cudaGetLastError();
     return nullptr;  // not cached: a later call retries
   }
@@ -110,7 +115,7 @@ const RouteDevice* route_device() {
 }
 
 template <int NB>
-tk_status launch_scatter(const tk_route_plan& pl, const tkg::RouteParams& p, cudaStream_t stream) {
+tk_status launch_scatter(const tk_route_plan& pl, const tkg::RouteParams& p, bool fused, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.ctas);
   cfg.blockDim = dim3(pl.threads);
@@ -126,15 +131,23 @@ tk_status launch_scatter(const tk_route_plan& pl, const tkg::RouteParams& p, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cudaError_t err;
   if (pl.ctas == 1)
-    return cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, true>, p) == cudaSuccess ? TK_OK : TK_ERR_CUDA;
-  return cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, false>, p) == cudaSuccess ? TK_OK : TK_ERR_CUDA;
+    err = cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, tkg::ROUTE_ONE_CTA>, p);
+  else if (fused)
+    err = cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, tkg::ROUTE_FUSED>, p);
+  else
+    err = cudaLaunchKernelEx(&cfg, tkg::route_scatter_kernel<NB, tkg::ROUTE_TABLE>, p);
+  return err == cudaSuccess ? TK_OK : TK_ERR_CUDA;
 }
 
 // The launches on `stream`: the scatter kernel alone for one CTA, else the
 // count kernel and the scatter kernel; `counts` holds plan.workspace_bytes.
+// fused: the gating launch before has filled the counts table (and `counts`
+// holds plan.fused_workspace_bytes: the table, then the arrival counter), so
+// only the scatter kernel runs.
 tk_status launch_route(const tk_route_plan& pl, const int32_t* ids, int64_t n, int32_t E, int32_t* counts,
-                       int32_t* offsets, int32_t* sorted_slots, int32_t* slot_pos, cudaStream_t stream) {
+                       int32_t* offsets, int32_t* sorted_slots, int32_t* slot_pos, bool fused, cudaStream_t stream) {
   tkg::RouteParams p;
   p.ids = ids;
   p.n = n;
@@ -144,13 +157,16 @@ tk_status launch_route(const tk_route_plan& pl, const int32_t* ids, int64_t n, i
   p.G = pl.ctas;
   p.warp_slots = pl.warp_slots;
   p.counts = counts;
+  p.done = fused && counts != nullptr
+               ? reinterpret_cast<uint32_t*>(counts + static_cast<int64_t>(pl.ctas) * p.E4)
+               : nullptr;
   p.offsets = offsets;
   p.sorted_slots = sorted_slots;
   p.slot_pos = slot_pos;
   p.err_word = tkg::device_error_word();
   if (p.err_word == nullptr) return TK_ERR_CUDA;
 
-  if (pl.ctas > 1) {
+  if (pl.ctas > 1 && !fused) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.ctas);
     cfg.blockDim = dim3(pl.threads);
@@ -163,10 +179,10 @@ tk_status launch_route(const tk_route_plan& pl, const int32_t* ids, int64_t n, i
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, tkg::route_count_kernel, p) != cudaSuccess) return TK_ERR_CUDA;
   }
-  if (E <= 16) return launch_scatter<4>(pl, p, stream);
-  if (E <= 64) return launch_scatter<6>(pl, p, stream);
-  if (E <= 256) return launch_scatter<8>(pl, p, stream);
-  return launch_scatter<10>(pl, p, stream);
+  if (E <= 16) return launch_scatter<4>(pl, p, fused, stream);
+  if (E <= 64) return launch_scatter<6>(pl, p, fused, stream);
+  if (E <= 256) return launch_scatter<8>(pl, p, fused, stream);
+  return launch_scatter<10>(pl, p, fused, stream);
 }
 
 tk_status route_checked(const int32_t* ids, int64_t T, int32_t k, int32_t E, int32_t* offsets,
@@ -225,6 +241,27 @@ int32_t* static_scratch() {
 
 }  // namespace
 
+namespace tkg {
+
+// The routing half of tk_gating_fused_topk_route (tk_gating.cu): validation and
+// the plan on the current device, then the placing launch after the gating.
+tk_status route_fused_plan(int64_t T, int32_t k, int32_t E, tk_route_plan* pl) {
+  const tk_status st = validate_route(T, k, E);
+  if (st != TK_OK) return st;
+  const RouteDevice* dev = route_device();
+  if (dev == nullptr) return TK_ERR_CUDA;
+  if (dev->status != TK_OK) return dev->status;
+  return route_plan_impl(T, k, E, dev->num_sms, pl);
+}
+
+tk_status route_fused_launch(const tk_route_plan& pl, const int32_t* ids, int64_t n, int32_t E, int32_t* workspace,
+                             int32_t* offsets, int32_t* sorted_slots, int32_t* slot_pos, cudaStream_t stream) {
+  return launch_route(pl, ids, n, E, pl.ctas > 1 ? workspace : nullptr, offsets, sorted_slots, slot_pos, pl.ctas > 1,
+                      stream);
+}
+
+}  // namespace tkg
+
 extern "C" {
 
 tk_status tk_gating_route_plan(int64_t T, int32_t k, int32_t E, int32_t num_sms, tk_route_plan* plan) {
@@ -239,14 +276,14 @@ tk_status tk_gating_route(const int32_t* ids, int64_t T, int32_t k, int32_t E, i
   if (st != TK_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (pl.workspace_bytes == 0)
-    return launch_route(pl, ids, T * static_cast<int64_t>(k), E, nullptr, offsets, sorted_slots, slot_pos, s);
+    return launch_route(pl, ids, T * static_cast<int64_t>(k), E, nullptr, offsets, sorted_slots, slot_pos, false, s);
   void* ws = nullptr;
   if (cudaMallocAsync(&ws, static_cast<size_t>(pl.workspace_bytes), s) != cudaSuccess) {
     cudaGetLastError();
     return TK_ERR_CUDA;
   }
   st = launch_route(pl, ids, T * static_cast<int64_t>(k), E, static_cast<int32_t*>(ws), offsets, sorted_slots,
-                    slot_pos, s);
+                    slot_pos, false, s);
   if (cudaFreeAsync(ws, s) != cudaSuccess && st == TK_OK) st = TK_ERR_CUDA;
   return st;
 }
@@ -261,7 +298,7 @@ tk_status tk_gating_route_static(const int32_t* ids, int64_t T, int32_t k, int32
   int32_t* scratch = static_scratch();
   if (scratch == nullptr) return TK_ERR_CUDA;
   return launch_route(pl, ids, T * static_cast<int64_t>(k), E, pl.workspace_bytes > 0 ? scratch : nullptr, offsets,
-                      sorted_slots, slot_pos, static_cast<cudaStream_t>(stream));
+                      sorted_slots, slot_pos, false, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

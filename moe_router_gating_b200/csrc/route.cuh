@@ -38,6 +38,13 @@ constexpr int ROUTE_THREADS = ROUTE_WARPS * 32;
 constexpr int ROUTE_MIN_WARP_SLOTS = 128;  // at least four 32-slot batches per warp
 constexpr int ROUTE_PREFETCH = 8;          // batches of ids in flight per warp
 
+// Where the placing kernel gets the per-CTA counts from.
+enum RouteMode : int {
+  ROUTE_ONE_CTA = 0,  // one CTA: it counts its own slots, no table
+  ROUTE_TABLE = 1,    // route_count_kernel wrote the table just before
+  ROUTE_FUSED = 2,    // the gating kernel added its ids to the table (route_counts.cuh)
+};
+
 struct RouteParams {
   const int32_t* ids;
   int64_t n;             // T * k
@@ -47,6 +54,7 @@ struct RouteParams {
   int32_t G;             // CTAs
   int64_t warp_slots;    // L: slots per warp range, a multiple of 32
   int32_t* counts;       // workspace [G][E4] (several CTAs only)
+  uint32_t* done;        // ROUTE_FUSED: CTAs that have read the table (zero between calls)
   int32_t* offsets;      // [E + 1]
   int32_t* sorted_slots; // [n]
   int32_t* slot_pos;     // [n]
@@ -225,7 +233,7 @@ __device__ __forceinline__ void route_table_sums(const RouteParams& p, int32_t* 
 //   below [E4]               counts over CTAs before this one
 //   part  [2][ROUTE_THREADS] int4 partial column sums (several CTAs only)
 //   warp_sums [ROUTE_WARPS + 1]
-template <int NB, bool SINGLE>
+template <int NB, int MODE>
 __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const RouteParams p) {
   extern __shared__ int32_t route_smem[];
   int32_t* base = route_smem;
@@ -235,18 +243,20 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
   int4* part = reinterpret_cast<int4*>(warp_sums + 36);  // 16-byte aligned: Ep*32 + 2*E4 + 36 is a multiple of 4
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31u;
+  __shared__ int route_flags[2];  // [0] this CTA's table row disagrees with its ids, [1] this CTA read the table last
 
-  // 1. this CTA's per-warp counts.  One CTA: this kernel is the programmatic
-  //    dependent of whatever precedes it and waits for it first.  Several: the
-  //    count kernel let this one start only after its own wait, so the ids are
-  //    complete and may be read before this kernel's dependency wait.
-  if (SINGLE) pdl_wait_primary();
+  // 1. this CTA's per-warp counts.  One CTA, or counts from the gating: this
+  //    kernel is the programmatic dependent of the kernel that wrote the ids (and
+  //    the table) and waits for it first.  Counts from route_count_kernel: that
+  //    kernel let this one start only after its own wait, so the ids are complete
+  //    and may be read before this kernel's dependency wait.
+  if (MODE != ROUTE_TABLE) pdl_wait_primary();
   int64_t beg, end;
   route_warp_range(p, &beg, &end);
   route_cta_warp_counts(p, base, beg, end);
 
   // 2. per-expert totals and the counts of earlier CTAs
-  if (SINGLE) {
+  if (MODE == ROUTE_ONE_CTA) {
     for (int e = threadIdx.x; e < p.E4; e += ROUTE_THREADS) {
       int32_t c = 0;
       if (e < p.E) {
@@ -258,8 +268,32 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
     }
     __syncthreads();
   } else {
-    pdl_wait_primary();  // the counts table is complete and visible
+    if (MODE == ROUTE_TABLE) pdl_wait_primary();  // the counts table is complete and visible
+    if (MODE == ROUTE_FUSED) {
+      // the gating's row of this CTA must equal what the CTA has just counted;
+      // it does unless the table was not zero before the gating launch
+      if (threadIdx.x == 0) route_flags[0] = 0;
+      __syncthreads();
+      const int32_t* row = p.counts + static_cast<int64_t>(blockIdx.x) * p.E4;
+      bool bad = false;
+      for (int e = threadIdx.x; e < p.E; e += ROUTE_THREADS) {
+        int32_t c = 0;
+#pragma unroll 8
+        for (int w = 0; w < ROUTE_WARPS; ++w) c += base[w * p.Ep + e];
+        bad |= __ldcg(row + e) != c;
+      }
+      if (bad) route_flags[0] = 1;
+    }
     route_table_sums(p, total, below, part);
+    if (MODE == ROUTE_FUSED) {
+      // every read of the table by this CTA is complete (route_table_sums ends
+      // with a CTA barrier); the CTA that reads it last zeroes it at the end
+      if (threadIdx.x == 0) {
+        if (route_flags[0] != 0) atomicOr(p.err_word, ERR_ROUTE_COUNTS);
+        __threadfence();
+        route_flags[1] = atomicAdd(p.done, 1u) == static_cast<uint32_t>(p.G - 1);
+      }
+    }
   }
 
   // 3. global offsets (every CTA forms them; CTA 0 stores them)
@@ -300,10 +334,26 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
       // the lowest lane of each group moves its expert's position past the group
       if (e[i] >= 0 && (grp & lt) == 0) my[e[i]] += __popc(grp);
       __syncwarp();
-      if (s < end && TK_CHECK(pos < p.n, p.err_word)) {
+      // counts from the gating are checked, not trusted: a position outside
+      // [0, n) is never written (ERR_ROUTE_COUNTS is set then)
+      const bool in_range = MODE == ROUTE_FUSED ? pos < p.n : TK_CHECK(pos < p.n, p.err_word);
+      if (s < end && in_range) {
         p.slot_pos[s] = pos;
         if (pos >= 0) p.sorted_slots[pos] = static_cast<int32_t>(s);
       }
+    }
+  }
+
+  // 6. counts from the gating: the last CTA to read the table leaves it zero for
+  //    the next call (the other CTAs read it before their arrival above)
+  if (MODE == ROUTE_FUSED) {
+    __syncthreads();
+    if (route_flags[1]) {
+      __threadfence();
+      int4* tab = reinterpret_cast<int4*>(p.counts);
+      const int64_t quads = static_cast<int64_t>(p.G) * (p.E4 / 4);
+      for (int64_t q = threadIdx.x; q < quads; q += ROUTE_THREADS) tab[q] = make_int4(0, 0, 0, 0);
+      if (threadIdx.x == 0) *p.done = 0u;
     }
   }
 }

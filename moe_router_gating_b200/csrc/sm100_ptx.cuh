@@ -29,6 +29,7 @@ enum : uint32_t {
   ERR_WAIT_DRAIN = 1u << 3,
   ERR_WAIT_CLUSTER = 1u << 4,
   ERR_BOUNDS = 1u << 5,  // debug builds: an index check failed; the access was skipped
+  ERR_ROUTE_COUNTS = 1u << 6,  // routing counts from the gating disagreed with the ids (table not zero before)
 };
 
 // Debug builds (compiled with -DTK_GATING_DEBUG, libtk_gating_debug.so): TK_CHECK

@@ -280,8 +280,11 @@ const DeviceState* device_state() {
   return &d;
 }
 
+// route: per-expert counts of the stored ids for the routing that follows
+// (tk_gating_fused_topk_route); a null table when nothing is counted.
 tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int64_t H, int64_t E, int32_t k,
-                            float* scores, int32_t* ids, float* logits, cudaStream_t stream) {
+                            float* scores, int32_t* ids, float* logits, cudaStream_t stream,
+                            const tkg::RouteCounts& route = tkg::RouteCounts{nullptr, 0u, 0}) {
   tk_status st = validate_sizes(T, H, E, k);
   if (st != TK_OK) return st;
   if (T == 0) return TK_OK;
@@ -303,7 +306,7 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
   const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
-                           dev->clock};
+                           dev->clock, route};
   return tkg::launch_planned<false>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, logits, stream);
 }
 
@@ -341,7 +344,7 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
       !encode_2d_u8(&mw, gate_q, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kslice, tkg::B_BOX_N))
     return TK_ERR_CUDA;
   const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
-                           dev->clock};
+                           dev->clock, tkg::RouteCounts{nullptr, 0u, 0}};
   return tkg::launch_planned<true>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, logits,
                                    stream);
 }
@@ -349,6 +352,11 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
 }  // namespace
 
 namespace tkg {
+// route.cu: the routing half of tk_gating_fused_topk_route
+tk_status route_fused_plan(int64_t T, int32_t k, int32_t E, tk_route_plan* pl);
+tk_status route_fused_launch(const tk_route_plan& pl, const int32_t* ids, int64_t n, int32_t E, int32_t* workspace,
+                             int32_t* offsets, int32_t* sorted_slots, int32_t* slot_pos, cudaStream_t stream);
+
 // The device error word of the current device for the other kernels of this
 // library (expert-parallel dispatch and combine); null without an sm_100 device.
 uint32_t* device_error_word() {
@@ -371,6 +379,36 @@ tk_status tk_gating_fused_topk_logits(const void* hidden, const void* gate_weigh
   if (logits == nullptr) return TK_ERR_INVALID_ARG;
   if (!aligned16(logits)) return TK_ERR_ALIGNMENT;
   return fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, logits, static_cast<cudaStream_t>(stream));
+}
+
+tk_status tk_gating_fused_topk_route(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,
+                                     int32_t k, float* scores, int32_t* ids, int32_t* offsets, int32_t* sorted_slots,
+                                     int32_t* slot_pos, void* workspace, int64_t workspace_bytes, void* stream) {
+  tk_status st = validate_sizes(T, H, E, k);
+  if (st != TK_OK) return st;
+  if (T > 0 && T > static_cast<int64_t>(INT32_MAX) / k) return TK_ERR_UNSUPPORTED;  // positions are int32
+  if (offsets == nullptr) return TK_ERR_INVALID_ARG;
+  if (T > 0 && (!hidden || !gate_weight || !scores || !ids || !sorted_slots || !slot_pos)) return TK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0 || (reinterpret_cast<uintptr_t>(sorted_slots) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(slot_pos) & 3u) != 0)
+    return TK_ERR_ALIGNMENT;
+  if (T > 0 && (!aligned16(hidden) || !aligned16(gate_weight) || !aligned16(scores) || !aligned16(ids)))
+    return TK_ERR_ALIGNMENT;
+  tk_route_plan rp;  // needs the device's SM count
+  st = tkg::route_fused_plan(T, k, static_cast<int32_t>(E), &rp);
+  if (st != TK_OK) return st;
+  if (rp.fused_workspace_bytes > 0) {
+    if (workspace == nullptr || workspace_bytes < rp.fused_workspace_bytes) return TK_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return TK_ERR_ALIGNMENT;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t E4 = static_cast<int32_t>((E + 3) / 4 * 4);
+  const tkg::RouteCounts rc{rp.ctas > 1 ? static_cast<int32_t*>(workspace) : nullptr,
+                            static_cast<uint32_t>(rp.warp_slots * (rp.threads / 32)), E4};  // a CTA's range: its warps' ranges
+  st = fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, nullptr, s, rc);
+  if (st != TK_OK) return st;
+  return tkg::route_fused_launch(rp, ids, T * static_cast<int64_t>(k), static_cast<int32_t>(E),
+                                 static_cast<int32_t*>(workspace), offsets, sorted_slots, slot_pos, s);
 }
 
 tk_status tk_gating_fused_topk_host(const void* hidden_host, const void* gate_weight, int64_t T, int64_t H,

@@ -239,3 +239,40 @@ def test_binding_rejects_bad_logits_before_the_call():
         _binding._check_logits(torch.empty((3, 4), dtype=torch.float64), 3, 4, torch.device("cpu"))
     _binding._check_logits(torch.empty((3, 4)), 3, 4, torch.device("cpu"))
 
+
+
+def test_fused_route_entry_point_rejects_before_cuda():
+    f = tk.fused_topk_gating_route_ptr
+    # (hidden, gate, T, H, E, k, scores, ids, offsets, sorted_slots, slot_pos, workspace, workspace_bytes)
+    ok = (16, 16, 8, 64, 16, 2, 16, 16, 16, 16, 16, 16, 1 << 20)
+
+    def call(**kw):
+        names = ("hidden", "gate", "T", "H", "E", "k", "scores", "ids", "offsets", "sorted_slots", "slot_pos",
+                 "workspace", "workspace_bytes")
+        args = dict(zip(names, ok))
+        args.update(kw)
+        return f(*(args[n] for n in names))
+
+    assert call(k=17) == tk.TK_ERR_INVALID_ARG           # k > E
+    assert call(E=1032) == tk.TK_ERR_UNSUPPORTED         # E > 1024
+    assert call(H=60) == tk.TK_ERR_UNSUPPORTED           # H % 8 != 0
+    assert call(T=1 << 28, k=8) == tk.TK_ERR_UNSUPPORTED  # T * k >= 2^31
+    assert call(offsets=0) == tk.TK_ERR_INVALID_ARG
+    assert call(sorted_slots=0) == tk.TK_ERR_INVALID_ARG
+    assert call(hidden=0) == tk.TK_ERR_INVALID_ARG
+    assert call(slot_pos=18) == tk.TK_ERR_ALIGNMENT      # routing outputs: 4-byte aligned
+    assert call(ids=20) == tk.TK_ERR_ALIGNMENT           # gating outputs: 16-byte aligned
+    # valid arguments without a GPU: no CPU fallback
+    assert call() in (tk.TK_ERR_CUDA, tk.TK_ERR_UNSUPPORTED)
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 8, 256), (512, 8, 256), (513, 8, 256), (65536, 8, 256), (3001, 16, 1024),
+                                   (12345, 7, 999)])
+def test_fused_route_workspace_is_the_table_and_a_counter(T, k, E):
+    p = tk.route_plan(T, k, E, 148)
+    if p["ctas"] == 1:
+        assert p["fused_workspace_bytes"] == 0
+    else:
+        assert p["fused_workspace_bytes"] == p["workspace_bytes"] + 16 == p["ctas"] * ((E + 3) // 4 * 4) * 4 + 16
+        # a gating row's k <= 32 assignments cross at most one routing range boundary
+        assert p["warp_slots"] * 32 >= 4096 >= k
