@@ -760,8 +760,12 @@ def run_route_ours(args, wl):
             return sum(a.elapsed_time(b) for a, b in evs) / args.steps
 
         gating_alone_ms = timed(lambda: tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream))
+        # the separate calls through the no-allocation routing entry point (the same
+        # kernels as tk_gating_route, without its stream-ordered workspace allocation)
         chained_ms = timed(lambda: (tk.fused_topk_gating(x, w, k, scores=scores, ids=ids, stream=stream),
-                                    tk.route(ids, E, offsets, sorted_slots, slot_pos, stream=stream)))
+                                    tk.route_static_ptr(ids.data_ptr(), T, k, E, offsets.data_ptr(),
+                                                        sorted_slots.data_ptr(), slot_pos.data_ptr(),
+                                                        stream.cuda_stream)))
 
     # end to end: pinned host ids -> device, route, the three outputs -> pinned host
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
@@ -809,6 +813,8 @@ def run_route_ours(args, wl):
         line["routing_added_us"] = (ms_per_step - gating_alone_ms) * 1e3
         line["separate_calls_ms_per_step"] = chained_ms
         line["separate_calls_routing_added_us"] = (chained_ms - gating_alone_ms) * 1e3
+        line["separate_calls_path"] = ("tk_gating_fused_topk, then tk_gating_route_static (count kernel + "
+                                       "placing kernel, no allocation)")
     if not chain:
         ach = bytes_alg / (ms_per_step / 1e3) / 1e9
         line["roofline"] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
