@@ -187,25 +187,37 @@ class ClockSampler:
         p, h = self._nvml, self._h
         power = None
         i = 0
+        self.query_s = []
         while not self._stop.is_set():
+            t0 = time.perf_counter()
             try:
                 sm = p.nvmlDeviceGetClockInfo(h, p.NVML_CLOCK_SM)
                 reasons = self._reasons(h)
                 if i % 8 == 0:
                     power = p.nvmlDeviceGetPowerUsage(h) / 1000.0
-                self.samples.append((sm, reasons, power))
+                if self._recording:
+                    self.samples.append((sm, reasons, power))
             except Exception as e:
                 self.error = repr(e)
+            self.query_s.append(time.perf_counter() - t0)
             i += 1
+            self._ready.set()
             self._stop.wait(self.period)
 
     def __enter__(self):
+        # the thread's first NVML queries (which may take milliseconds) run before
+        # the timed region; only samples taken inside it are kept
+        self._recording = False
+        self._ready = threading.Event()
         if self._nvml is not None:
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
+            self._ready.wait(1.0)
+        self._recording = True
         return self
 
     def __exit__(self, *exc):
+        self._recording = False
         self._stop.set()
         if self._thread is not None:
             self._thread.join()
@@ -229,7 +241,17 @@ class ClockSampler:
             "power_w_max": max([s[2] for s in self.samples if s[2] is not None], default=None),
             "source": "NVML (same counters as nvidia-smi), sampled every %.1f ms during the timed region"
                       % (self.period * 1e3),
+            "nvml_query_ms_median": (statistics.median(self.query_s[1:]) * 1e3
+                                     if len(getattr(self, "query_s", [])) > 1 else None),
         }
+
+
+def wait_releasing_gil(event) -> None:
+    """Wait for `event` by polling with short sleeps, so that the clock sampler's
+    thread gets the interpreter while the timed launches run (a blocking
+    synchronize may hold it); the caller still synchronizes afterwards."""
+    while not event.query():
+        time.sleep(0.0002)
 
 
 # ---------------------------------------------------------------------------
@@ -354,6 +376,7 @@ def run_ours(args, wl):
             for _ in range(args.steps):
                 step()
             ev1.record(stream)
+            wait_releasing_gil(ev1)
             torch.cuda.synchronize(dev)
             elapsed_ms = ev0.elapsed_time(ev1)
             launch_ms = elapsed_ms / args.steps
@@ -366,6 +389,7 @@ def run_ours(args, wl):
                 a.record(stream)
                 step()
                 b.record(stream)
+            wait_releasing_gil(evs[-1][1])
             torch.cuda.synchronize(dev)
             per = [a.elapsed_time(b) for a, b in evs]
             elapsed_ms = sum(per)
