@@ -47,9 +47,13 @@
 //               (measured ~15% faster than one slice per stage on the 65536-token
 //               workload).
 //   warps 2..5  epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (one token row
-//               per thread), keeps a running top-k, applies the softmax and
-//               stores.  The accumulator is double-buffered in tensor memory, so
-//               the epilogue of one tile overlaps the MMAs of the next.
+//   (or 2..9)   per thread), keeps a running top-k, applies the softmax and
+//               stores.  With eight epilogue warps (epi_warps), warps 2..5 take
+//               the first half of a tile's expert columns and warps 6..9 the
+//               second; the second half's lists go through shared memory to the
+//               first half's threads, which merge them before the softmax.  The
+//               accumulator is double-buffered in tensor memory, so the epilogue
+//               of one tile overlaps the MMAs of the next.
 #pragma once
 
 #include <cuda.h>
@@ -68,9 +72,22 @@ constexpr int UMMA_K = 16;                              // K per tcgen05.mma (ki
 constexpr int A_STAGE_BYTES = BLOCK_M * BLOCK_K * 2;    // 16 KB hidden slice
 constexpr int B_BOX_N = 64;                             // experts per gate box
 constexpr int B_BOX_BYTES = BLOCK_K * B_BOX_N * 2;      // 8 KB gate box
-constexpr int NUM_EPI_WARPS = 4;
+constexpr int EPI_BARRIER_RESERVE = 256;                // barriers and flags after the ring (bytes)
 constexpr int KB_PER_STAGE = 2;                         // 64-wide K slices per ring stage
-constexpr int ROW_TILE_THREADS = 64 + NUM_EPI_WARPS * 32;
+
+// Epilogue warps of a kernel instance: one per tensor-memory lane quadrant, or
+// two (each taking half of a tile's expert columns) where the selection is the
+// larger cost -- lists of 16 or 32, or two expert groups per tile.  Measured on
+// one B200 (outputs bitwise equal): 65536 x 2048 x 256 with k = 16 92.8 vs 111.6
+// us, 20000 x 2048 x 512 FP8 with k = 32 140 vs 196 us, 20000 x 2048 x 1024 with
+// k = 8 122-127 vs 129-140 us; with k <= 8 and one group no gain (train shape
+// 199.7-204.6 vs 198.7-201.3 us), so those keep four.
+__host__ __device__ constexpr int epi_warps(int kmax, int expert_groups) {
+  return (kmax >= 16 || expert_groups == 2) ? 8 : 4;
+}
+__host__ __device__ constexpr int row_tile_threads(int kmax, int expert_groups) {
+  return 64 + 32 * epi_warps(kmax, expert_groups);
+}
 
 constexpr int N_CHUNK = 256;                            // MMA N per instruction (chunk of experts)
 
@@ -249,10 +266,11 @@ __device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (
 // group bookkeeping: kept at run time it cost ~4% of the 65536-token kernel's
 // cycles).
 template <int KMAX, int CG, bool FP8, int EG>
-__global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
+__global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
     gating_row_tiles_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_x64,
                             const __grid_constant__ CUtensorMap map_w, const RowTileParams p) {
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
+  constexpr int NUM_EPI_WARPS = epi_warps(KMAX, EG);
   constexpr bool kPair = CG == 2;
   const bool clock_cta = p.clock != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
   const uint64_t t0_ns = clock_cta ? globaltimer_ns() : 0;
@@ -268,6 +286,11 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // eight epilogue warps: hand-over of the second column half's lists of a full
+  // tile, 128 rows of KMAX values, then of KMAX ids (the host adds its bytes to
+  // the launch's shared memory)
+  float* hand_v = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + EPI_BARRIER_RESERVE);
+  int32_t* hand_i = reinterpret_cast<int32_t*>(hand_v + BLOCK_M * KMAX);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -472,7 +495,8 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
     __syncwarp();
   } else {
     // ---------------- epilogue ----------------
-    const int quad = warp & 3;  // TMEM lanes this warp may access
+    const int quad = warp & 3;       // TMEM lanes this warp may access
+    const int hc = (warp - 2) >> 2;  // column half of this warp (0: warps 2..5, 1: warps 6..9)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     int local = 0;
     TileWork w;
@@ -510,10 +534,15 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           ncols = min(chunk_n(gs, c) / 2, p.E - col_base);
           chunk_addr += static_cast<uint32_t>(c * N_CHUNK);
         }
+        // this warp's half of the pass's columns: [0, mid) or [mid, ncols), mid a
+        // multiple of 32 (one tensor-memory load)
+        const int mid = NUM_EPI_WARPS == 4 ? ncols : min(ncols, (ncols + 63) / 64 * 32);
+        const int lo = hc == 0 ? 0 : mid;
+        const int hi = hc == 0 ? mid : ncols;
         // 64 columns per round trip: two loads, one wait
-        for (int c0 = 0; c0 < ncols; c0 += 64) {
+        for (int c0 = lo; c0 < hi; c0 += 64) {
           uint32_t r0[32], r1[32];
-          const bool second = c0 + 32 < ncols;  // warp-uniform
+          const bool second = c0 + 32 < hi;  // warp-uniform
           // the columns read stay inside this CTA's tensor-memory allocation
           if (!TK_CHECK(((chunk_addr - tmem_base) & 0xFFFFu) + c0 + (second ? 64u : 32u) <= p.tmem_cols, p.err_word))
             break;
@@ -521,12 +550,12 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
           if (second) tmem_ld_32(chunk_addr + c0 + 32, r1);
           tmem_ld_wait();
           scale_chunk<FP8>(r0, p.gscale, col_base + c0, p.E, hs);
-          if (dump) store_logit_chunk(p.logits, my_row, p.E, col_base + c0, col_base + ncols, r0);
-          offer_chunk(top, r0, c0, ncols, col_base);
+          if (dump) store_logit_chunk(p.logits, my_row, p.E, col_base + c0, col_base + hi, r0);
+          offer_chunk(top, r0, c0, hi, col_base);
           if (second) {
             scale_chunk<FP8>(r1, p.gscale, col_base + c0 + 32, p.E, hs);
-            if (dump) store_logit_chunk(p.logits, my_row, p.E, col_base + c0 + 32, col_base + ncols, r1);
-            offer_chunk(top, r1, c0 + 32, ncols, col_base);
+            if (dump) store_logit_chunk(p.logits, my_row, p.E, col_base + c0 + 32, col_base + hi, r1);
+            offer_chunk(top, r1, c0 + 32, hi, col_base);
           }
         }
       }
@@ -543,37 +572,68 @@ __global__ void __launch_bounds__(ROW_TILE_THREADS, 1)
 
       if (w.eg + 1 < EG) continue;  // the tile's next expert group follows
       if (!w.half) {
-        const int64_t row = static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
-        if (row < p.T) {
-          top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
-          if (p.route.table != nullptr) route_count_row(p.route, top, p.k, row, p.E);
+        // the second half's list of each row goes to the first half's thread of
+        // that row (the next tile's lists are written only after every epilogue
+        // warp has passed the next tile's agreement barrier, i.e. after these reads)
+        if constexpr (NUM_EPI_WARPS == 8) {
+          float* xv = hand_v + (quad * 32 + lane) * KMAX;
+          int32_t* xi = hand_i + (quad * 32 + lane) * KMAX;
+          if (hc == 1) {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+              xv[j] = top.v[j];
+              xi[j] = top.i[j];
+            }
+          }
+          named_barrier_sync(3, NUM_EPI_WARPS * 32);
+          if (hc == 0) {
+            float bv[KMAX];
+            int32_t bi[KMAX];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+              bv[j] = xv[j];
+              bi[j] = xi[j];
+            }
+            merge_sorted(top, bv, bi);
+          }
+        }
+        if (hc == 0) {
+          const int64_t row = static_cast<int64_t>(w.row0) + rank * BLOCK_M + quad * 32 + lane;
+          if (row < p.T) {
+            top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);
+            if (p.route.table != nullptr) route_count_row(p.route, top, p.k, row, p.E);
+          }
         }
       } else {
         // A half tile is a CTA's last tile (and this its last expert group), so
-        // its ring is idle: the upper lanes
-        // hand their lists to the lower lanes of the same rows through it.
+        // its ring is idle: each of a row's four lists (lane half x column half)
+        // but the lower lanes' first half goes through it to that thread.
         const int m = (quad & 1) * 32 + lane;  // row within this CTA's 64
-        // the hand-over area (64 rows of KMAX floats, then of KMAX ids) lies inside the idle ring
-        if (!TK_CHECK(BLOCK_M * KMAX * 8 <= p.stages * KB_PER_STAGE * A_STAGE_BYTES, p.err_word)) break;
-        float* xv = reinterpret_cast<float*>(sA) + m * KMAX;
-        int32_t* xi = reinterpret_cast<int32_t*>(sA + BLOCK_M * KMAX * 4) + m * KMAX;
-        if (upper) {
+        const int slot = (upper ? 2 : 0) + hc;  // this thread's list of row m
+        // the hand-over area (64 rows x 4 lists of KMAX floats, then of KMAX ids) lies inside the idle ring
+        if (!TK_CHECK(4 * (BLOCK_M / 2) * KMAX * 8 <= p.stages * KB_PER_STAGE * A_STAGE_BYTES, p.err_word)) break;
+        float* xv = reinterpret_cast<float*>(sA) + m * 4 * KMAX;
+        int32_t* xi = reinterpret_cast<int32_t*>(sA + 4 * (BLOCK_M / 2) * KMAX * 4) + m * 4 * KMAX;
+        if (slot != 0) {
 #pragma unroll
           for (int j = 0; j < KMAX; ++j) {
-            xv[j] = top.v[j];
-            xi[j] = top.i[j];
+            xv[slot * KMAX + j] = top.v[j];
+            xi[slot * KMAX + j] = top.i[j];
           }
         }
         named_barrier_sync(1, NUM_EPI_WARPS * 32);
-        if (!upper) {
-          float bv[KMAX];
-          int32_t bi[KMAX];
+        if (slot == 0) {
+          for (int o = 1; o < 4; ++o) {
+            if (NUM_EPI_WARPS == 4 && (o & 1)) continue;  // four warps: no second column half
+            float bv[KMAX];
+            int32_t bi[KMAX];
 #pragma unroll
-          for (int j = 0; j < KMAX; ++j) {
-            bv[j] = xv[j];
-            bi[j] = xi[j];
+            for (int j = 0; j < KMAX; ++j) {
+              bv[j] = xv[o * KMAX + j];
+              bi[j] = xi[o * KMAX + j];
+            }
+            merge_sorted(top, bv, bi);
           }
-          merge_sorted(top, bv, bi);
           const int64_t row = static_cast<int64_t>(w.row0) + rank * (BLOCK_M / 2) + m;
           if (row < p.T) {
             top.softmax_store(p.k, p.scores + row * p.k, p.ids + row * p.k);

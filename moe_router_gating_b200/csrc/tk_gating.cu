@@ -25,7 +25,7 @@ __device__ uint64_t g_tk_clock[3] = {0, 0, 0};
 std::atomic<uint64_t> g_timeout_ns{1000000000ull};
 
 constexpr int kMaxDynamicSmem = tkg::kMaxDynamicSmem;
-constexpr int kSmemReserve = 1024 + 256;  // 1 KB alignment pad + barriers and flags
+constexpr int kSmemReserve = 1024 + tkg::EPI_BARRIER_RESERVE;  // 1 KB alignment pad + barriers and flags
 constexpr int kMaxStages = 8;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -134,7 +134,12 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   const int acc_bufs = 2 * acc_stride <= 512 ? 2 : 1;  // 512 tensor-memory columns
   const int b_boxes = pair ? g_pad / 2 / tkg::B_BOX_N : (g_pad + tkg::B_BOX_N - 1) / tkg::B_BOX_N;
   const int stage_bytes = tkg::KB_PER_STAGE * (tkg::A_STAGE_BYTES + b_boxes * tkg::B_BOX_BYTES);
-  int stages = (kMaxDynamicSmem - kSmemReserve) / stage_bytes;
+  // eight epilogue warps: the hand-over of one column half's top-k lists, 128 rows of
+  // KMAX (value, id) pairs
+  const int kmax = k <= 4 ? 4 : (k <= 8 ? 8 : (k <= 16 ? 16 : 32));
+  const int groups = n_pad > tkg::E_GROUP ? 2 : 1;
+  const int hand_bytes = tkg::epi_warps(kmax, groups) == 8 ? tkg::BLOCK_M * kmax * 8 : 0;
+  int stages = (kMaxDynamicSmem - kSmemReserve - hand_bytes) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return TK_ERR_UNSUPPORTED;
   const int64_t rows_per_tile = static_cast<int64_t>(tkg::BLOCK_M) * cg;
@@ -165,8 +170,8 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   plan->grid = static_cast<int32_t>(units * cg);
   plan->num_half_tiles = static_cast<int32_t>(half_tiles);
   plan->cluster = cg;
-  plan->threads = tkg::ROW_TILE_THREADS;
-  plan->smem_bytes = stages * stage_bytes + kSmemReserve;
+  plan->threads = tkg::row_tile_threads(kmax, groups);
+  plan->smem_bytes = stages * stage_bytes + kSmemReserve + hand_bytes;
   plan->tmem_cols = static_cast<int32_t>(pow2_at_least(acc_bufs * acc_stride));
   plan->slices_per_stage = tkg::KB_PER_STAGE;
   plan->expert_groups = n_pad > tkg::E_GROUP ? 2 : 1;
