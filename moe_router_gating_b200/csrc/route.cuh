@@ -183,8 +183,10 @@ __device__ __forceinline__ int32_t route_block_exclusive_scan(int32_t* v, int32_
 
 // Column sums of the counts table: total[e] over all CTAs, below[e] over the
 // CTAs before this one.  `part` holds 2 * ROUTE_THREADS int4 of scratch.
+// own_row (optional, E4 words of shared memory) receives this CTA's own row of
+// the table as it goes by.
 __device__ __forceinline__ void route_table_sums(const RouteParams& p, int32_t* total, int32_t* below,
-                                                 int4* part) {
+                                                 int4* part, int32_t* own_row = nullptr) {
   const int quads = p.E4 / 4;
   const int groups = ROUTE_THREADS / quads;  // row groups (quads <= ROUTE_THREADS)
   const int q = threadIdx.x % quads;
@@ -202,6 +204,8 @@ __device__ __forceinline__ void route_table_sums(const RouteParams& p, int32_t* 
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
+        if (own_row != nullptr && r + u * groups == static_cast<int>(blockIdx.x))
+          reinterpret_cast<int4*>(own_row)[q] = v[u];
         sa.x += v[u].x; sa.y += v[u].y; sa.z += v[u].z; sa.w += v[u].w;
         if (r + u * groups < static_cast<int>(blockIdx.x)) {
           sb.x += v[u].x; sb.y += v[u].y; sb.z += v[u].z; sb.w += v[u].w;
@@ -244,6 +248,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31u;
   __shared__ int route_flags[2];  // [0] this CTA's table row disagrees with its ids, [1] this CTA read the table last
+  // counts from the gating: this CTA's row of the table, kept from the column sums' pass
+  __shared__ __align__(16) int32_t own_row[MODE == ROUTE_FUSED ? TK_ROUTE_MAX_EXPERTS : 4];
 
   // 1. this CTA's per-warp counts.  One CTA, or counts from the gating: this
   //    kernel is the programmatic dependent of the kernel that wrote the ids (and
@@ -269,35 +275,45 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
     __syncthreads();
   } else {
     if (MODE == ROUTE_TABLE) pdl_wait_primary();  // the counts table is complete and visible
+    if (MODE == ROUTE_FUSED && threadIdx.x == 0) route_flags[0] = 0;
+    route_table_sums(p, total, below, part, MODE == ROUTE_FUSED ? own_row : nullptr);
     if (MODE == ROUTE_FUSED) {
+      // every read of the table by this CTA is complete (route_table_sums ends
+      // with a CTA barrier): count the arrival; the CTA that arrives last zeroes
+      // the table right after the scan below (its fence here orders those stores
+      // after every other CTA's reads, which preceded their arrivals)
+      if (threadIdx.x == 0) {
+        __threadfence();
+        const bool last = atomicAdd(p.done, 1u) == static_cast<uint32_t>(p.G - 1);
+        if (last) __threadfence();
+        route_flags[1] = last;
+      }
       // the gating's row of this CTA must equal what the CTA has just counted;
       // it does unless the table was not zero before the gating launch
-      if (threadIdx.x == 0) route_flags[0] = 0;
-      __syncthreads();
-      const int32_t* row = p.counts + static_cast<int64_t>(blockIdx.x) * p.E4;
       bool bad = false;
       for (int e = threadIdx.x; e < p.E; e += ROUTE_THREADS) {
         int32_t c = 0;
 #pragma unroll 8
         for (int w = 0; w < ROUTE_WARPS; ++w) c += base[w * p.Ep + e];
-        bad |= __ldcg(row + e) != c;
+        bad |= own_row[e] != c;
       }
       if (bad) route_flags[0] = 1;
-    }
-    route_table_sums(p, total, below, part);
-    if (MODE == ROUTE_FUSED) {
-      // every read of the table by this CTA is complete (route_table_sums ends
-      // with a CTA barrier); the CTA that reads it last zeroes it at the end
-      if (threadIdx.x == 0) {
-        if (route_flags[0] != 0) atomicOr(p.err_word, ERR_ROUTE_COUNTS);
-        __threadfence();
-        route_flags[1] = atomicAdd(p.done, 1u) == static_cast<uint32_t>(p.G - 1);
-      }
     }
   }
 
   // 3. global offsets (every CTA forms them; CTA 0 stores them)
-  const int32_t placed = route_block_exclusive_scan(total, p.E, warp_sums);
+  const int32_t placed = route_block_exclusive_scan(total, p.E, warp_sums);  // (its barriers also publish route_flags)
+  if (MODE == ROUTE_FUSED) {
+    if (threadIdx.x == 0 && route_flags[0] != 0) atomicOr(p.err_word, ERR_ROUTE_COUNTS);
+    // every CTA has read the table: the last one to arrive leaves it zero for the
+    // next call (while the other CTAs place their slots)
+    if (route_flags[1]) {
+      int4* tab = reinterpret_cast<int4*>(p.counts);
+      const int64_t quads = static_cast<int64_t>(p.G) * (p.E4 / 4);
+      for (int64_t q = threadIdx.x; q < quads; q += ROUTE_THREADS) tab[q] = make_int4(0, 0, 0, 0);
+      if (threadIdx.x == 0) *p.done = 0u;
+    }
+  }
   if (blockIdx.x == 0) {
     for (int e = threadIdx.x; e < p.E; e += ROUTE_THREADS) p.offsets[e] = total[e];
     if (threadIdx.x == 0) p.offsets[p.E] = placed;
@@ -341,19 +357,6 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_scatter_kernel(const Rout
         p.slot_pos[s] = pos;
         if (pos >= 0) p.sorted_slots[pos] = static_cast<int32_t>(s);
       }
-    }
-  }
-
-  // 6. counts from the gating: the last CTA to read the table leaves it zero for
-  //    the next call (the other CTAs read it before their arrival above)
-  if (MODE == ROUTE_FUSED) {
-    __syncthreads();
-    if (route_flags[1]) {
-      __threadfence();
-      int4* tab = reinterpret_cast<int4*>(p.counts);
-      const int64_t quads = static_cast<int64_t>(p.G) * (p.E4 / 4);
-      for (int64_t q = threadIdx.x; q < quads; q += ROUTE_THREADS) tab[q] = make_int4(0, 0, 0, 0);
-      if (threadIdx.x == 0) *p.done = 0u;
     }
   }
 }
