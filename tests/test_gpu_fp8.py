@@ -47,6 +47,8 @@ def check_fp8(wl, duplicate_pairs=(), rows=None):
     (20000, 512, 256, 8), (19999, 512, 200, 8), (16384, 4096, 64, 6), (30000, 256, 512, 32), (1000, 1024, 512, 16),
     (3, 2048, 64, 4), (129, 144, 24, 5), (200, 512, 1024, 8), (20000, 256, 768, 8), (300, 256, 1024, 32),
     (24000, 128, 1016, 32),
+    # eight epilogue warps: one CTA per tile (E <= 64, k = 16) and pairs with half tiles (k = 16)
+    (20000, 512, 64, 16), (40000, 512, 256, 16),
 ])
 def test_fp8_shapes(T, H, E, k):
     check_fp8(workloads.RouterWorkload(f"fp8_{T}_{H}_{E}_{k}", T, H, E, k, seed=7))

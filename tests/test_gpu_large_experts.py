@@ -36,6 +36,8 @@ def clean_error_word():
     (300, 256, 1024, 32), (24000, 128, 1016, 32),
     # k up to 32 with one chunk
     (2000, 1024, 256, 32), (40000, 512, 256, 32), (5000, 256, 64, 32), (700, 256, 32, 32),
+    # one CTA per 128-token tile (E <= 64) with eight epilogue warps (lists of 16 and 32)
+    (20000, 512, 64, 16), (20011, 512, 64, 32), (12000, 256, 48, 24),
 ])
 def test_large_expert_shapes(T, H, E, k):
     check_workload(workloads.RouterWorkload(f"large_{T}_{H}_{E}_{k}", T, H, E, k, seed=5))
