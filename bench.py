@@ -60,6 +60,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workspace", action="store_true",
+                    help="time tk_gating_fused_topk (no workspace) instead of tk_gating_fused_topk_ws, whose many-token "
+                         "launches split their last round between CTA pairs")
     ap.add_argument("--no-workload-summary", action="store_true",
                     help="skip the per-workload table (every router workload, GPU and oracle, one GPU only)")
     ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (profiling cases)")
@@ -335,16 +338,21 @@ def run_ours(args, wl):
         wqd, wsd = torch.from_numpy(wq).to(dev), torch.from_numpy(ws).to(dev)
         hidden_bytes = wl.T * wl.H + 4 * wl.T
 
+        work = None if args.no_workspace else tk.gating_workspace(wl.T, wl.H, wl.E, wl.k, dev, fp8=True)
+
         def gate(xx):
-            return lambda: tk.fused_topk_gating_fp8(xx, xsd, wqd, wsd, wl.k, scores=scores, ids=ids, stream=stream)
+            return lambda: tk.fused_topk_gating_fp8(xx, xsd, wqd, wsd, wl.k, scores=scores, ids=ids, stream=stream,
+                                                    workspace=work)
     else:
         x_host = workloads.to_torch_bf16(rank_wl.hidden())
         w = workloads.to_torch_bf16(rank_wl.gate_weight()).to(dev)
         x = x_host.to(dev)
         hidden_bytes = wl.T * wl.H * 2
 
+        work = None if args.no_workspace else tk.gating_workspace(wl.T, wl.H, wl.E, wl.k, dev)
+
         def gate(xx):
-            return lambda: tk.fused_topk_gating(xx, w, wl.k, scores=scores, ids=ids, stream=stream)
+            return lambda: tk.fused_topk_gating(xx, w, wl.k, scores=scores, ids=ids, stream=stream, workspace=work)
     big = hidden_bytes > L2_BYTES
     # 16 MB up to L2: back-to-back launches over rotating hidden buffers that together
     # exceed twice L2 (each launch reads a hidden tensor evicted since its last use)
@@ -449,8 +457,10 @@ def run_ours(args, wl):
     roofline["traffic"] = traffic
     roofline.update({"traffic_source": traffic_src, "kernel_source_digest": digest})
 
-    plan = tk.make_plan(wl.T, wl.H // 2 if fp8 else wl.H, wl.E, wl.k,
-                        torch.cuda.get_device_properties(dev).multi_processor_count)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    plan_h = wl.H // 2 if fp8 else wl.H
+    plan = tk.make_plan(wl.T, plan_h, wl.E, wl.k, sms) if args.no_workspace else \
+        tk.make_plan_ws(wl.T, plan_h, wl.E, wl.k, sms)[0]
 
     cpu = None
     if not args.no_cpu_baseline and world == 1 and not fp8:
@@ -481,6 +491,7 @@ def run_ours(args, wl):
                   "L2 flushed (256 MB write) before every timed launch; each launch timed alone",
             "parallelism": "single GPU" if world == 1 else f"{world} ranks, independent token shards, no collective",
             "launch": plan,
+            "entry": "tk_gating_fused_topk" if args.no_workspace else "tk_gating_fused_topk_ws",
         },
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -632,8 +643,10 @@ def per_workload_summary(dev, peaks, peak_src, cpu_seconds: float, with_cpu: boo
         big = hidden_bytes > L2_BYTES
         rotate = not big and hidden_bytes >= 16 * 1024 * 1024
 
+        work = tk.gating_workspace(wl.T, wl.H, wl.E, wl.k, dev)
+
         def gate(xx):
-            return lambda: tk.fused_topk_gating(xx, w, wl.k, scores=s, ids=i, stream=stream)
+            return lambda: tk.fused_topk_gating(xx, w, wl.k, scores=s, ids=i, stream=stream, workspace=work)
         flushed_ms = None
         if not big:
             tk.clock_counters(clear=True)
@@ -664,9 +677,11 @@ def per_workload_summary(dev, peaks, peak_src, cpu_seconds: float, with_cpu: boo
                               "roofline_frac_sustained": roof["roofline_frac_sustained"],
                               "roofline_us": roof["roofline_us"]},
                  "sm_mhz_in_kernel": clk["sm_ghz"] * 1e3 if clk["sm_ghz"] else None,
-                 "plan": {k: v for k, v in tk.make_plan(wl.T, wl.H, wl.E, wl.k,
-                                                        torch.cuda.get_device_properties(dev).multi_processor_count)
-                          .items() if k in ("variant", "cluster", "grid", "num_tiles", "num_half_tiles")}}
+                 "plan": {k: v for k, v in tk.make_plan_ws(wl.T, wl.H, wl.E, wl.k,
+                                                           torch.cuda.get_device_properties(dev).multi_processor_count)[0]
+                          .items() if k in ("variant", "cluster", "grid", "num_tiles", "num_half_tiles",
+                                            "num_split_tiles")},
+                 "entry": "tk_gating_fused_topk_ws"}
         if err := tk.device_error(clear=True):
             raise SystemExit(f"device error word {err:#x} during the {name} summary")
         if with_cpu:

@@ -193,6 +193,9 @@ typedef struct {
   int32_t num_half_tiles; /* CTA pairs: 128-token tiles after the full ones (balanced last round) */
   int32_t slices_per_stage; /* 64-wide K slices per ring stage */
   int32_t expert_groups;  /* groups of at most 512 experts, computed one after the other per tile (1 or 2) */
+  int32_t num_split_tiles; /* workspace entry points: last-round 256-token tiles each split in H between two
+                              CTA pairs, in place of the half tiles (0: none) */
+  int32_t split_k_block;   /* the K slice (of 64) at which a split tile's H range is cut */
 } tk_gating_plan;
 
 /*
@@ -204,6 +207,88 @@ typedef struct {
  * Validates like tk_gating_fused_topk (pointers excepted).  Makes no CUDA call.
  */
 TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan);
+
+/*
+ * tk_gating_fused_topk_ws -- tk_gating_fused_topk with a caller-owned device
+ * workspace, which lets the many-token launch end its last round sooner.
+ *
+ * The operation, outputs and errors are those of tk_gating_fused_topk
+ * (section 4.1, "MoE Gating"); only the schedule of the last round differs.
+ * Where the plan without workspace ends with a round of 128-token "half" tiles
+ * on CTA pairs (many tokens, 64 < E <= 512, k <= 8), this call instead cuts
+ * each of the last round's 256-token tiles in H between two CTA pairs: the
+ * first accumulates H slices [0, split_k_block) of the tile and stores its
+ * fp32 accumulator rows to the workspace, the second accumulates the rest,
+ * adds the stored rows to its own (first half + second half, fp32) and selects,
+ * applies the softmax and stores as tk_gating_fused_topk does.  A split tile
+ * costs about half of a full tile where a half tile costs ~0.9.  The logits
+ * of those rows are therefore fp32 sums in a different association; selections
+ * agree wherever the k-th and (k+1)-th logits are not within fp32 rounding.
+ * Elsewhere the launch is tk_gating_fused_topk's and the workspace untouched.
+ *
+ *   workspace        device, 16-byte aligned, at least the bytes that
+ *                    tk_gating_workspace_bytes (or tk_gating_make_plan_ws)
+ *                    gives for this call (8.9 MB at T = 65536, E = 256,
+ *                    k = 8 on a B200); may be NULL when that is 0.  It starts
+ *                    with flags (8 bytes per split tile, rounded up to 256)
+ *                    that must be zero before the first call: zero the
+ *                    workspace once after allocating it; every
+ *                    call leaves them zero, so calls in order on one stream
+ *                    may share a workspace.  Calls that may run at the same
+ *                    time need workspaces of their own.  After a call that
+ *                    reported an expired wait (tk_gating_device_error), zero
+ *                    it again.
+ *   workspace_bytes  its size.
+ *   the other arguments as tk_gating_fused_topk.
+ *
+ * The second half's pair waits (bounded, as every wait in the kernels) for
+ * the first half's rows; both are CTAs of the same launch, which fits one
+ * wave.  Errors: those of tk_gating_fused_topk, and TK_ERR_INVALID_ARG when
+ * the workspace is NULL or smaller than needed (or workspace_bytes < 0),
+ * TK_ERR_ALIGNMENT when it is not 16-byte aligned.  Allocates nothing.
+ */
+TK_API tk_status tk_gating_fused_topk_ws(const void* hidden, const void* gate_weight, int64_t T, int64_t H,
+                                         int64_t E, int32_t k, float* scores, int32_t* ids, void* workspace,
+                                         int64_t workspace_bytes, void* stream);
+
+/*
+ * tk_gating_fused_topk_fp8_ws -- tk_gating_fused_topk_fp8 with a workspace, as
+ * tk_gating_fused_topk_ws: the stored first half is the unscaled fp32 sum of
+ * E4M3 products; the second half's pair scales each summed logit by
+ * gate_scale[e] and then hidden_scale[t], as tk_gating_fused_topk_fp8 does.
+ */
+TK_API tk_status tk_gating_fused_topk_fp8_ws(const void* hidden_q, const float* hidden_scale, const void* gate_q,
+                                             const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k,
+                                             float* scores, int32_t* ids, void* workspace, int64_t workspace_bytes,
+                                             void* stream);
+
+/*
+ * tk_gating_fused_topk_ws_logits -- tk_gating_fused_topk_ws that also stores
+ * every logit its selection ranked into logits (device, fp32 [T, E], 16-byte
+ * aligned), as tk_gating_fused_topk_logits does.  A verification aid.
+ */
+TK_API tk_status tk_gating_fused_topk_ws_logits(const void* hidden, const void* gate_weight, int64_t T, int64_t H,
+                                                int64_t E, int32_t k, float* scores, int32_t* ids, float* logits,
+                                                void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
+ * tk_gating_make_plan_ws -- the launch tk_gating_fused_topk_ws makes for
+ * (T, H, E, k) on a device like tk_gating_make_plan's, and the workspace bytes
+ * it needs (0 when the launch is the one without workspace).  For the FP8
+ * entry point pass H / 2.  Makes no CUDA call.
+ */
+TK_API tk_status tk_gating_make_plan_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
+                                        tk_gating_plan* plan, int64_t* workspace_bytes);
+
+/*
+ * tk_gating_workspace_bytes -- the workspace bytes tk_gating_fused_topk_ws
+ * (fp8 = 0) or tk_gating_fused_topk_fp8_ws (fp8 != 0) needs for (T, H, E, k)
+ * on the current device.  Validates the sizes like those calls.  Errors:
+ * TK_ERR_INVALID_ARG for a null result pointer, the size errors, and
+ * TK_ERR_CUDA / TK_ERR_UNSUPPORTED without an sm_100 device.
+ */
+TK_API tk_status tk_gating_workspace_bytes(int64_t T, int64_t H, int64_t E, int32_t k, int32_t fp8,
+                                           int64_t* workspace_bytes);
 
 /*
  * tk_gating_device_error -- read the device error word of the current device

@@ -30,9 +30,12 @@ from ._binding import (  # noqa: F401
     fused_topk_gating_ptr,
     fused_topk_gating_route,
     fused_topk_gating_route_ptr,
+    fused_topk_gating_ws_ptr,
+    gating_workspace,
     library,
     library_path,
     make_plan,
+    make_plan_ws,
     route,
     route_plan,
     route_ptr,
@@ -40,11 +43,13 @@ from ._binding import (  # noqa: F401
     route_static_ptr,
     set_wait_timeout_ns,
     status_string,
+    workspace_bytes,
 )
 
 __all__ = [
     "fused_topk_gating", "fused_topk_gating_fp8", "fused_topk_gating_host", "fused_topk_gating_ptr",
     "fused_topk_gating_route", "fused_topk_gating_route_ptr", "route_workspace", "make_plan", "route", "route_plan",
+    "fused_topk_gating_ws_ptr", "gating_workspace", "workspace_bytes", "make_plan_ws",
     "route_ptr", "route_static_ptr", "device_error", "clock_counters",
     "set_wait_timeout_ns", "status_string", "TkGatingError", "library", "library_path",
 ]

@@ -34,7 +34,8 @@ class TkGatingError(RuntimeError):
 class _Plan(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in (
         "variant", "block_m", "n_pad", "num_tiles", "k_blocks", "split_h", "stages", "grid", "cluster",
-        "threads", "smem_bytes", "tmem_cols", "num_half_tiles", "slices_per_stage", "expert_groups")]
+        "threads", "smem_bytes", "tmem_cols", "num_half_tiles", "slices_per_stage", "expert_groups",
+        "num_split_tiles", "split_k_block")]
 
 
 class _RoutePlan(ctypes.Structure):
@@ -66,6 +67,17 @@ def library() -> ctypes.CDLL:
             lib.tk_gating_fused_topk_fp8.restype = ctypes.c_int
             lib.tk_gating_fused_topk_route.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, i64, vp]
             lib.tk_gating_fused_topk_route.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_ws.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, i64, vp]
+            lib.tk_gating_fused_topk_ws.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_ws_logits.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, i64, vp]
+            lib.tk_gating_fused_topk_ws_logits.restype = ctypes.c_int
+            lib.tk_gating_fused_topk_fp8_ws.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, i64, vp]
+            lib.tk_gating_fused_topk_fp8_ws.restype = ctypes.c_int
+            lib.tk_gating_make_plan_ws.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(_Plan),
+                                                   ctypes.POINTER(ctypes.c_int64)]
+            lib.tk_gating_make_plan_ws.restype = ctypes.c_int
+            lib.tk_gating_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_int64)]
+            lib.tk_gating_workspace_bytes.restype = ctypes.c_int
             lib.tk_gating_fused_topk_logits.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
             lib.tk_gating_fused_topk_logits.restype = ctypes.c_int
             lib.tk_gating_fused_topk_fp8_logits.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
@@ -119,14 +131,61 @@ def fused_topk_gating_ptr(hidden: int, gate_weight: int, T: int, H: int, E: int,
     return int(library().tk_gating_fused_topk(hidden, gate_weight, T, H, E, k, scores, ids, stream))
 
 
-def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, stream=None, logits=None):
+def fused_topk_gating_ws_ptr(hidden: int, gate_weight: int, T: int, H: int, E: int, k: int, scores: int, ids: int,
+                             workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    """Raw C-ABI call of the workspace entry point (integer device pointers);
+    returns the tk_status."""
+    return int(library().tk_gating_fused_topk_ws(hidden, gate_weight, T, H, E, k, scores, ids, workspace,
+                                                 workspace_bytes, stream))
+
+
+def workspace_bytes(T: int, H: int, E: int, k: int, fp8: bool = False) -> int:
+    """Bytes of workspace the workspace entry points need for (T, H, E, k) on the
+    current device (0 where they make the launch without one)."""
+    n = ctypes.c_int64(0)
+    _check(library().tk_gating_workspace_bytes(T, H, E, k, 1 if fp8 else 0, ctypes.byref(n)),
+           "tk_gating_workspace_bytes")
+    return int(n.value)
+
+
+def gating_workspace(T: int, H: int, E: int, k: int, device=None, fp8: bool = False):
+    """A zeroed uint8 CUDA tensor (at least 256 bytes) to serve as the
+    ``workspace`` of ``fused_topk_gating`` / ``fused_topk_gating_fp8`` for
+    (T, H, E, k) on ``device``; every call leaves it ready for the next one on
+    the same stream.  Calls that may overlap on the device need their own."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        n = workspace_bytes(T, H, E, k, fp8)
+    return torch.zeros(max(256, n), dtype=torch.uint8, device=dev)
+
+
+def make_plan_ws(T: int, H: int, E: int, k: int, num_sms: int = 148) -> tuple[dict, int]:
+    """The launch of the workspace entry point and its workspace bytes (host logic only)."""
+    p = _Plan()
+    n = ctypes.c_int64(0)
+    _check(library().tk_gating_make_plan_ws(T, H, E, k, num_sms, ctypes.byref(p), ctypes.byref(n)),
+           "tk_gating_make_plan_ws")
+    return {name: getattr(p, name) for name, _ in _Plan._fields_}, int(n.value)
+
+
+def _check_workspace(workspace, device) -> None:
+    if not workspace.is_cuda or workspace.device != device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor on the inputs' device")
+
+
+def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, stream=None, logits=None,
+                      workspace=None):
     """``(scores[T,k] fp32, ids[T,k] int32) = softmax(topk(hidden @ gate_weight))``.
 
     ``hidden`` is a CUDA bf16 ``[T, H]`` tensor and ``gate_weight`` a CUDA bf16
     ``[H, E]`` tensor, both contiguous.  Output tensors may be passed in.  The
     launch goes on ``stream`` (default: the current torch stream).  Passing a
     contiguous fp32 ``[T, E]`` CUDA tensor as ``logits`` calls the verification
-    entry point, which also stores every logit the selection ranked.
+    entry point, which also stores every logit the selection ranked.  Passing a
+    ``workspace`` (from ``gating_workspace``) calls the workspace entry point,
+    whose last round of a many-token launch splits its tiles in H between CTA
+    pairs.
     """
     import torch
     if hidden.dtype != torch.bfloat16 or gate_weight.dtype != torch.bfloat16:
@@ -153,6 +212,11 @@ def fused_topk_gating(hidden, gate_weight, top_k: int, scores=None, ids=None, st
         _check_logits(logits, T, E, hidden.device)
         args = args + (logits.data_ptr(),)
         fn, name = lib.tk_gating_fused_topk_logits, "tk_gating_fused_topk_logits"
+    if workspace is not None:
+        _check_workspace(workspace, hidden.device)
+        args = args + (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        fn, name = ((lib.tk_gating_fused_topk_ws_logits, "tk_gating_fused_topk_ws_logits") if logits is not None
+                    else (lib.tk_gating_fused_topk_ws, "tk_gating_fused_topk_ws"))
     if hidden.device.index == torch.cuda.current_device():
         st = fn(*args, _stream_handle(stream, hidden.device))
     else:
@@ -249,12 +313,14 @@ def fused_topk_gating_fp8_ptr(hidden_q: int, hidden_scale: int, gate_q: int, gat
 
 
 def fused_topk_gating_fp8(hidden_q, hidden_scale, gate_q, gate_scale, top_k: int, scores=None, ids=None,
-                          stream=None, logits=None):
+                          stream=None, logits=None, workspace=None):
     """Fused gating on FP8 E4M3 inputs: ``hidden_q`` [T, H] and ``gate_q`` [E, H]
     (expert-major) as torch.float8_e4m3fn or torch.uint8 CUDA tensors, with fp32
     ``hidden_scale`` [T] and ``gate_scale`` [E].  Returns ``(scores, ids)``.
     ``logits`` (fp32 [T, E]) selects the verification entry point, which also
-    stores every scaled logit the selection ranked."""
+    stores every scaled logit the selection ranked; ``workspace`` (from
+    ``gating_workspace(..., fp8=True)``) the workspace entry point (not
+    combined with ``logits``)."""
     import torch
     fp8_types = (torch.float8_e4m3fn, torch.uint8)
     if hidden_q.dtype not in fp8_types or gate_q.dtype not in fp8_types:
@@ -277,10 +343,16 @@ def fused_topk_gating_fp8(hidden_q, hidden_scale, gate_q, gate_scale, top_k: int
     args = (hidden_q.data_ptr(), hidden_scale.data_ptr(), gate_q.data_ptr(), gate_scale.data_ptr(), T, H, E,
             int(top_k), scores.data_ptr(), ids.data_ptr())
     fn, name = library().tk_gating_fused_topk_fp8, "tk_gating_fused_topk_fp8"
+    if logits is not None and workspace is not None:
+        raise ValueError("the FP8 workspace entry point has no logits variant")
     if logits is not None:
         _check_logits(logits, T, E, hidden_q.device)
         args = args + (logits.data_ptr(),)
         fn, name = library().tk_gating_fused_topk_fp8_logits, "tk_gating_fused_topk_fp8_logits"
+    if workspace is not None:
+        _check_workspace(workspace, hidden_q.device)
+        args = args + (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        fn, name = library().tk_gating_fused_topk_fp8_ws, "tk_gating_fused_topk_fp8_ws"
     with torch.cuda.device(hidden_q.device):
         st = fn(*args, _stream_handle(stream, hidden_q.device))
     _check(st, name)

@@ -29,7 +29,22 @@ struct LaunchEnv {
   uint64_t timeout_ns;    // bounded-wait limit
   uint64_t* clock;        // SM-clock counters of the launches (cycles, ns, launches)
   RouteCounts route;      // per-expert counts of the stored ids by routing range; table null: none
+  void* workspace;        // split last round (plan.num_split_tiles > 0): flags, then first-half partials
+  uint32_t split_token;   // non-zero, different for every launch
 };
+
+// Workspace of a split last round: num_split x 2 uint32 flags (8 bytes per tile,
+// rounded up to 256), then the first halves' fp32 rows, num_split x 256 rows of
+// round_up(E, 32) + 4 floats (the 4 keep consecutive rows off the same
+// shared-memory banks once copied there).
+inline int split_part_cols(int64_t E) { return round_up(static_cast<int>(E), 32); }
+inline int split_part_stride(int64_t E) { return split_part_cols(E) + 4; }
+inline int64_t split_flag_bytes(int num_split) { return (static_cast<int64_t>(num_split) * 8 + 255) / 256 * 256; }
+inline int64_t split_workspace_bytes(int num_split, int64_t E) {
+  return num_split > 0
+             ? split_flag_bytes(num_split) + static_cast<int64_t>(num_split) * 256 * split_part_stride(E) * 4
+             : 0;
+}
 
 // Shared-memory limits (and non-portable cluster sizes) of every kernel instance
 // of one precision; once per device.

@@ -17,6 +17,7 @@ template <int KMAX, bool FP8>
 bool set_up_kernels_of() {
   bool ok = set_smem_limit(gating_row_tiles_kernel<KMAX, 1, FP8, 1>) &&
             set_smem_limit(gating_row_tiles_kernel<KMAX, 2, FP8, 1>) &&
+            (KMAX > 8 || set_smem_limit(gating_row_tiles_kernel<(KMAX > 8 ? 8 : KMAX), 2, FP8, 1, true>)) &&
             set_smem_limit(gating_row_tiles_kernel<KMAX, 2, FP8, 2>) &&
             set_smem_limit(gating_split_h_kernel<KMAX, 2, FP8>) &&
             set_smem_limit(gating_split_h_kernel<KMAX, 4, FP8>) &&
@@ -32,10 +33,10 @@ bool set_up_gating_kernels() {
          set_up_kernels_of<32, FP8>();
 }
 
-template <int KMAX, int CG, bool FP8, int EG>
+template <int KMAX, int CG, bool FP8, int EG, bool SPLIT = false>
 tk_status launch_row_tiles(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
                            const CUtensorMap& mw, const RowTileParams& prm, cudaStream_t stream) {
-  auto kernel = gating_row_tiles_kernel<KMAX, CG, FP8, EG>;
+  auto kernel = gating_row_tiles_kernel<KMAX, CG, FP8, EG, SPLIT>;
   // programmatic dependent launch: CTAs may start on SMs the previous kernel has
   // left and set up while it finishes (the producer waits before its loads)
   cudaLaunchAttribute attr[2];
@@ -97,6 +98,11 @@ tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, co
                              const CUtensorMap& mw, const RowTileParams& prm, cudaStream_t stream) {
   if (pl.variant == TK_VARIANT_ROW_PAIRS) {
     if (pl.expert_groups == 2) return launch_row_tiles<KMAX, 2, FP8, 2>(pl, mx, mx64, mw, prm, stream);
+    if constexpr (KMAX <= 8) {
+      if (pl.num_split_tiles > 0) return launch_row_tiles<KMAX, 2, FP8, 1, true>(pl, mx, mx64, mw, prm, stream);
+    } else {
+      if (pl.num_split_tiles > 0) return TK_ERR_UNSUPPORTED;  // the planner splits only lists of <= 8
+    }
     return launch_row_tiles<KMAX, 2, FP8, 1>(pl, mx, mx64, mw, prm, stream);
   }
   return launch_row_tiles<KMAX, 1, FP8, 1>(pl, mx, mx64, mw, prm, stream);
@@ -168,6 +174,19 @@ tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const C
   prm.logits = logits;
   prm.clock = env.clock;
   prm.route = env.route;
+  prm.num_split = pl.num_split_tiles;
+  prm.split_kb = pl.split_k_block;
+  prm.part_cols = split_part_cols(E);
+  prm.part_stride = split_part_stride(E);
+  prm.split_token = env.split_token;
+  prm.split_flags = nullptr;
+  prm.split_part = nullptr;
+  if (pl.num_split_tiles > 0) {
+    if (env.workspace == nullptr) return TK_ERR_INVALID_ARG;
+    prm.split_flags = static_cast<uint32_t*>(env.workspace);
+    prm.split_part = reinterpret_cast<float*>(static_cast<uint8_t*>(env.workspace) +
+                                              split_flag_bytes(pl.num_split_tiles));
+  }
 
   if (k <= 4) return launch_row_variant<4, FP8>(pl, mx, mx64, mw, prm, stream);
   if (k <= 8) return launch_row_variant<8, FP8>(pl, mx, mx64, mw, prm, stream);

@@ -90,6 +90,7 @@ __host__ __device__ constexpr int row_tile_threads(int kmax, int expert_groups) 
 }
 
 constexpr int N_CHUNK = 256;                            // MMA N per instruction (chunk of experts)
+constexpr int XPOSE_STRIDE = 36;                        // floats per row of a warp's 32 x 32 store tile (16-byte rows)
 
 struct RowTileParams {
   int32_t T, H, E, k;
@@ -112,6 +113,21 @@ struct RowTileParams {
   float* logits;        // optional [T, E]: every logit the selection ranks is also stored (verification)
   uint64_t* clock;      // SM-clock counters: the first CTA adds its cycles and ns (and 1) per launch
   RouteCounts route;    // optional per-expert counts of the stored ids by routing range (route_counts.cuh)
+  // Split last round (pairs with one expert group and four epilogue warps, the
+  // workspace entry points): instead of half tiles, num_split 256-token tiles
+  // after the full ones, each cut in H at K slice split_kb between two pairs.
+  // Pair 2j ("first half") accumulates slices [0, split_kb) of split tile j and
+  // stores its fp32 accumulator rows to split_part[j][256 rows][part_stride], then
+  // sets split_flags[2j + CTA rank] = split_token; pair 2j + 1 accumulates the
+  // rest, waits for that flag, adds the stored partial to its own (first half +
+  // second half) and selects; it then clears the flag.
+  int32_t num_split;
+  int32_t split_kb;
+  int32_t part_cols;      // E rounded up to 32
+  int32_t part_stride;    // floats between stored rows: part_cols + 4 (rows 16 bytes off the banks' period)
+  uint32_t split_token;   // non-zero, different for every launch
+  float* split_part;
+  uint32_t* split_flags;
 };
 
 // K elements of H per K slice: one 128-byte swizzle row of bf16 or of FP8 values.
@@ -215,17 +231,34 @@ struct TileWork {
   int row0;   // first token row of the tile (pair tile: of the pair)
   bool half;  // 128-token pair tile
   int eg;     // expert group of this work item
+  int kb0;    // K slices [kb0, kb1) of this item: all of H unless split
+  int kb1;
+  int split;  // 0: a whole tile; 1 / 2: the first / second H half of split tile `sidx`
+  int sidx;
 };
 
-template <int CG, int EG>
+template <int CG, int EG, bool SPLIT>
 __device__ __forceinline__ bool tile_work(const RowTileParams& p, int unit, int units, int item, TileWork& w) {
   // every tile is EG (1 or 2) consecutive work items, one per expert group
   const int i = EG == 1 ? item : item >> 1;
   w.eg = EG == 1 ? 0 : item & 1;
+  w.kb0 = 0;
+  w.kb1 = p.k_blocks;
+  w.split = 0;
+  w.sidx = 0;
   const int n_full = unit < p.num_tiles ? (p.num_tiles - 1 - unit) / units + 1 : 0;
   if (i < n_full) {
     w.row0 = (unit + i * units) * (BLOCK_M * CG);
     w.half = false;
+    return true;
+  }
+  if (SPLIT && i == n_full && unit < 2 * p.num_split) {
+    w.sidx = unit >> 1;
+    w.split = 1 + (unit & 1);
+    w.row0 = (p.num_tiles + w.sidx) * (BLOCK_M * CG);
+    w.half = false;
+    w.kb0 = w.split == 1 ? 0 : p.split_kb;
+    w.kb1 = w.split == 1 ? p.split_kb : p.k_blocks;
     return true;
   }
   if (CG == 2 && i == n_full && unit < p.num_half) {
@@ -262,15 +295,53 @@ __device__ __forceinline__ void offer_chunk(RowTopK<KMAX>& top, const uint32_t (
   }
 }
 
+// Split last round: wait (one thread) until *flag == want, bounded like the
+// mbarrier waits; false (abort flag and error bit set) when the limit expires
+// or the CTA has already aborted.
+__device__ __forceinline__ bool wait_split_flag(const uint32_t* flag, uint32_t want, volatile int* abort,
+                                                uint64_t timeout_ns, uint32_t* err_word) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == want) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort = 1;
+      atomicOr(err_word, ERR_WAIT_EPILOGUE);
+      return false;
+    }
+    __nanosleep(256);
+  }
+}
+
+// r[j] <- other[j] + r[j] for the 32 floats of a chunk (the first H half's
+// partial, staged in shared memory, plus this CTA's own, in that order).
+__device__ __forceinline__ void add_first_half(uint32_t (&r)[32], const float* other) {
+  const float4* o = reinterpret_cast<const float4*>(other);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 v = o[q];
+    r[4 * q + 0] = __float_as_uint(v.x + __uint_as_float(r[4 * q + 0]));
+    r[4 * q + 1] = __float_as_uint(v.y + __uint_as_float(r[4 * q + 1]));
+    r[4 * q + 2] = __float_as_uint(v.z + __uint_as_float(r[4 * q + 2]));
+    r[4 * q + 3] = __float_as_uint(v.w + __uint_as_float(r[4 * q + 3]));
+  }
+}
+
 // EG: expert groups (compile time, so that the single-group kernel carries no
 // group bookkeeping: kept at run time it cost ~4% of the 65536-token kernel's
 // cycles).
-template <int KMAX, int CG, bool FP8, int EG>
+// SPLIT: the workspace entry points' split last round (pairs, one expert group,
+// four epilogue warps; RowTileParams::num_split): compiled into instances of
+// its own, so the other instances carry none of its code.
+template <int KMAX, int CG, bool FP8, int EG, bool SPLIT = false>
 __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
     gating_row_tiles_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_x64,
                             const __grid_constant__ CUtensorMap map_w, const RowTileParams p) {
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
   constexpr int NUM_EPI_WARPS = epi_warps(KMAX, EG);
+  static_assert(!SPLIT || (CG == 2 && EG == 1 && NUM_EPI_WARPS == 4), "split last round: pairs, one group, four warps");
   constexpr bool kPair = CG == 2;
   const bool clock_cta = p.clock != nullptr && blockIdx.x == 0 && threadIdx.x == 0;
   const uint64_t t0_ns = clock_cta ? globaltimer_ns() : 0;
@@ -286,6 +357,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  uint64_t* split_bar = reinterpret_cast<uint64_t*>(tmem_holder + 2);  // split second half: the partial's bulk load
   // eight epilogue warps: hand-over of the second column half's lists of a full
   // tile, 128 rows of KMAX values, then of KMAX ids (the host adds its bytes to
   // the launch's shared memory)
@@ -309,6 +381,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
       mbar_init(&acc_empty[b], NUM_EPI_WARPS * CG);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain, 1);
+    mbar_init(split_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&map_x);
@@ -350,7 +423,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
       int issued = 0;
       bool ok = true;
       TileWork w;
-      for (int item = 0; ok && tile_work<CG, EG>(p, unit, units, item, w); ++item) {
+      for (int item = 0; ok && tile_work<CG, EG, SPLIT>(p, unit, units, item, w); ++item) {
         const int cta_rows = w.half ? BLOCK_M / 2 : BLOCK_M;  // hidden rows this CTA stages
         const int row0 = w.row0 + static_cast<int>(rank) * cta_rows;
         // this work item's gate boxes: box j of a K slice starts at expert
@@ -365,7 +438,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
         const uint32_t stage_tx = KB_PER_STAGE * CG * (cta_rows * BLOCK_K * 2 + boxes * B_BOX_BYTES);
         const CUtensorMap* map_a = w.half ? &map_x64 : &map_x;
         // K slices past H (when k_blocks is odd) are out of bounds: TMA fills zeros
-        for (int kb = 0; kb < p.k_blocks; kb += KB_PER_STAGE) {
+        for (int kb = w.kb0; kb < w.kb1; kb += KB_PER_STAGE) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_PRODUCER, p.err_word)) {
             ok = false;
             break;
@@ -423,7 +496,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
       bool ok = true;
       int local = 0;
       TileWork w;
-      for (; ok && tile_work<CG, EG>(p, unit, units, local, w); ++local) {
+      for (; ok && tile_work<CG, EG, SPLIT>(p, unit, units, local, w); ++local) {
         const uint32_t buf = static_cast<uint32_t>(local % p.acc_bufs);
         const uint32_t acc_phase = static_cast<uint32_t>(local / p.acc_bufs) & 1;
         // this work item's chunks: instruction descriptors (pairs: M = 128 for a
@@ -437,7 +510,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
         if (!mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + buf * p.acc_stride;
-        for (int kb = 0; kb < p.k_blocks; kb += KB_PER_STAGE) {
+        for (int kb = w.kb0; kb < w.kb1; kb += KB_PER_STAGE) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.timeout_ns, ERR_WAIT_MMA, p.err_word)) {
             ok = false;
             break;
@@ -453,7 +526,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
             if (two_chunks) {
 #pragma unroll
               for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
-                const uint32_t accumulate = ((kb + sub) | kk) != 0;
+                const uint32_t accumulate = ((kb - w.kb0 + sub) | kk) != 0;
                 const uint64_t a_desc = a_desc_k_slice(a_addr, kk);
                 umma<FP8, kPair>(d_tmem, a_desc, gate_desc_k_slice<FP8>(b_addr, kk), id0, accumulate);
                 umma<FP8, kPair>(d_tmem + N_CHUNK, a_desc, gate_desc_k_slice<FP8>(b_addr + b_off1, kk), id1,
@@ -462,7 +535,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
             } else {
 #pragma unroll
               for (int kk = 0; kk < BLOCK_K / UMMA_K; ++kk) {
-                const uint32_t accumulate = ((kb + sub) | kk) != 0;
+                const uint32_t accumulate = ((kb - w.kb0 + sub) | kk) != 0;
                 umma<FP8, kPair>(d_tmem, a_desc_k_slice(a_addr, kk), gate_desc_k_slice<FP8>(b_addr, kk), id0,
                                  accumulate);
               }
@@ -501,7 +574,7 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
     int local = 0;
     TileWork w;
     RowTopK<KMAX> top;
-    for (; tile_work<CG, EG>(p, unit, units, local, w); ++local) {
+    for (; tile_work<CG, EG, SPLIT>(p, unit, units, local, w); ++local) {
       const uint32_t buf = static_cast<uint32_t>(local % p.acc_bufs);
       const uint32_t acc_phase = static_cast<uint32_t>(local / p.acc_bufs) & 1;
       const bool ok = mbar_wait(&acc_full[buf], acc_phase, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
@@ -510,6 +583,91 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
       // tile's list exchange below.
       if (!named_barrier_and(2, NUM_EPI_WARPS * 32, ok)) break;
       tc_fence_after_sync();
+
+      // split last round (pairs, one expert group, four epilogue warps)
+      const float* first_half = nullptr;  // second H half: the stored first-half partial of this thread's row
+      if constexpr (SPLIT) {
+        if (w.split == 1) {
+          // First H half: this CTA's 128 accumulator rows, columns [0, part_cols)
+          // (column c = expert c), to the workspace.  As in a half tile, this is
+          // the CTA's last item and its ring is idle: each warp moves its 32 rows
+          // in 32-column chunks through a padded tile there, so that every store
+          // instruction writes four whole 128-byte rows of a chunk.
+          const uint32_t acc_addr = lane_base + buf * p.acc_stride;
+          float* xpose = reinterpret_cast<float*>(sA) + quad * (32 * XPOSE_STRIDE);
+          const int row_in_tile = rank * BLOCK_M + quad * 32;  // this warp's first row of the 256
+          const int64_t row_base = static_cast<int64_t>(w.row0) + row_in_tile;
+          float* dst = p.split_part + (static_cast<int64_t>(w.sidx) * (2 * BLOCK_M) + row_in_tile) * p.part_stride;
+          const int qc = 4 * (lane & 7);
+          if (TK_CHECK(NUM_EPI_WARPS * 32 * XPOSE_STRIDE * 4 <= p.stages * KB_PER_STAGE * A_STAGE_BYTES, p.err_word)) {
+            for (int c0 = 0; c0 < p.part_cols; c0 += 32) {
+              uint32_t r[32];
+              if (!TK_CHECK(((acc_addr - tmem_base) & 0xFFFFu) + c0 + 32u <= p.tmem_cols, p.err_word)) break;
+              tmem_ld_32(acc_addr + c0, r);
+              tmem_ld_wait();
+              float* mine = xpose + lane * XPOSE_STRIDE;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(mine + j) = make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                                                   __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+              __syncwarp();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int rr = 4 * i + (lane >> 3);
+                const float4 v = *reinterpret_cast<const float4*>(xpose + rr * XPOSE_STRIDE + qc);
+                if (row_base + rr < p.T)
+                  *reinterpret_cast<float4*>(dst + static_cast<int64_t>(rr) * p.part_stride + c0 + qc) = v;
+              }
+              __syncwarp();
+            }
+          }
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) {
+            if (!leader)
+              mbar_arrive_remote(map_shared_rank(smem_u32(&acc_empty[buf]), 0));
+            else
+              mbar_arrive(&acc_empty[buf]);
+          }
+          // every warp's rows are stored: publish them to the second half's pair
+          named_barrier_sync(4, NUM_EPI_WARPS * 32);
+          if (warp == 2 && lane == 0) {
+            __threadfence();
+            atomicExch(p.split_flags + 2 * w.sidx + rank, p.split_token);
+          }
+          continue;
+        }
+        if (w.split == 2) {
+          // Second H half: wait until the first half's pair has stored the same
+          // rows (one thread polls, bounded; the warps agree on the outcome)
+          // This CTA's 128 rows of the first half are contiguous in the workspace:
+          // one bulk copy brings them into the idle ring (this is the CTA's last
+          // item), where each thread then reads its row.
+          const uint32_t rows_bytes = static_cast<uint32_t>(BLOCK_M * p.part_stride * 4);
+          bool got = true;
+          if (warp == 2 && lane == 0) {
+            got = wait_split_flag(p.split_flags + 2 * w.sidx + rank, p.split_token, abort_flag, p.timeout_ns,
+                                  p.err_word);
+            // the rows land in the idle ring (its hidden-row and gate parts together)
+            if (got && TK_CHECK(rows_bytes <= static_cast<uint32_t>(p.stages * KB_PER_STAGE *
+                                                                    (A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES)),
+                                p.err_word)) {
+              mbar_arrive_expect_tx(split_bar, rows_bytes);
+              bulk_load_g2s(sA,
+                            p.split_part + (static_cast<int64_t>(w.sidx) * (2 * BLOCK_M) + rank * BLOCK_M) * p.part_stride,
+                            rows_bytes, split_bar);
+            } else {
+              got = false;
+            }
+          }
+          got = named_barrier_and(4, NUM_EPI_WARPS * 32, got);
+          if (got) {
+            got = mbar_wait(split_bar, 0, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
+            got = named_barrier_and(4, NUM_EPI_WARPS * 32, got);
+          }
+          if (got) first_half = reinterpret_cast<const float*>(sA) + (quad * 32 + lane) * p.part_stride;
+        }
+      }
 
       // full tile: one row per thread, TMEM column c = expert e0 + c of the group;
       // half tile: per chunk c, lanes 0..63 hold experts e0 + [256c, 256c + N_c/2)
@@ -549,6 +707,12 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
           tmem_ld_32(chunk_addr + c0, r0);
           if (second) tmem_ld_32(chunk_addr + c0 + 32, r1);
           tmem_ld_wait();
+          if constexpr (SPLIT) {
+            if (first_half != nullptr) {  // split second half: add the first half's partial (full tiles: c = column)
+              add_first_half(r0, first_half + c0);
+              if (second) add_first_half(r1, first_half + c0 + 32);
+            }
+          }
           scale_chunk<FP8>(r0, p.gscale, col_base + c0, p.E, hs);
           if (dump) store_logit_chunk(p.logits, my_row, p.E, col_base + c0, col_base + hi, r0);
           offer_chunk(top, r0, c0, hi, col_base);
@@ -570,6 +734,13 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
           mbar_arrive(&acc_empty[buf]);
       }
 
+      if constexpr (SPLIT) {
+        if (w.split == 2) {
+          // every warp has read the first half's partial: clear the flag for the next call
+          named_barrier_sync(4, NUM_EPI_WARPS * 32);
+          if (warp == 2 && lane == 0 && first_half != nullptr) atomicExch(p.split_flags + 2 * w.sidx + rank, 0u);
+        }
+      }
       if (w.eg + 1 < EG) continue;  // the tile's next expert group follows
       if (!w.half) {
         // the second half's list of each row goes to the first half's thread of

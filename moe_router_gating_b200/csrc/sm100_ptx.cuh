@@ -182,6 +182,16 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Plain (untiled) bulk copy of `bytes` contiguous bytes from global memory into
+// this CTA's shared memory, completing on `bar`; both addresses 16-byte aligned,
+// `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // Same load for a CTA pair (tcgen05 cta_group::2): `bar_cluster_addr` may be the
 // mbarrier of the pair's leader CTA (shared::cluster address from mapa), so the
 // leader's barrier counts the bytes both CTAs load.  No multicast.

@@ -178,6 +178,31 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   return TK_OK;
 }
 
+// The plan of the workspace entry points (tk_gating_fused_topk_ws): the plan
+// without workspace, except that a last round of half tiles on CTA pairs (one
+// expert group, lists of at most 8) becomes ceil(half tiles / 2) 256-token tiles
+// each split in H between two pairs; *workspace_bytes is what that needs (0 when
+// nothing is split).
+tk_status plan_impl_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, const ClusterCapacity& cap,
+                       tk_gating_plan* plan, int64_t* workspace_bytes) {
+  if (workspace_bytes == nullptr) return TK_ERR_INVALID_ARG;
+  *workspace_bytes = 0;
+  const tk_status st = plan_impl(T, H, E, k, num_sms, cap, plan);
+  if (st != TK_OK) return st;
+  // measured: the split pays where the tiles are long (H >= 4096) and the first
+  // half's 128 KB per CTA fits the idle ring (E <= 256)
+  if (plan->variant != TK_VARIANT_ROW_PAIRS || plan->expert_groups != 1 || k > 8 || plan->num_half_tiles == 0 ||
+      plan->k_blocks < 64 || E > 256)
+    return TK_OK;
+  const int split = (plan->num_half_tiles + 1) / 2;  // 256-token tiles; at most half the pairs take one each
+  if (2 * split > plan->grid / 2) return TK_OK;
+  plan->num_split_tiles = split;
+  plan->split_k_block = round_up((plan->k_blocks + 1) / 2, tkg::KB_PER_STAGE);
+  plan->num_half_tiles = 0;
+  *workspace_bytes = tkg::split_workspace_bytes(split, E);
+  return TK_OK;
+}
+
 // ---- driver entry point for tensor-map encoding (no link-time libcuda) ----
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -285,11 +310,40 @@ const DeviceState* device_state() {
   return &d;
 }
 
+// A caller's workspace for the workspace entry points (null: the entry points
+// without one).
+struct Workspace {
+  void* ptr;
+  int64_t bytes;
+};
+
+// Launch tokens of split last rounds: non-zero, different for every launch.
+std::atomic<uint32_t> g_split_token{0};
+uint32_t next_split_token() {
+  uint32_t t = g_split_token.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (t == 0) t = g_split_token.fetch_add(1, std::memory_order_relaxed) + 1;
+  return t;
+}
+
+// Plan on the current device: without a workspace, or the workspace plan, whose
+// bytes the caller's workspace must hold (checked before any launch).
+tk_status plan_for_call(int64_t T, int64_t H, int64_t E, int32_t k, const DeviceState* dev, const Workspace* ws,
+                        tk_gating_plan* pl) {
+  if (ws == nullptr) return plan_impl(T, H, E, k, dev->num_sms, dev->capacity, pl);
+  int64_t need = 0;
+  const tk_status st = plan_impl_ws(T, H, E, k, dev->num_sms, dev->capacity, pl, &need);
+  if (st != TK_OK) return st;
+  if (need > 0 && (ws->ptr == nullptr || ws->bytes < need)) return TK_ERR_INVALID_ARG;
+  if (need > 0 && !aligned16(ws->ptr)) return TK_ERR_ALIGNMENT;
+  return TK_OK;
+}
+
 // route: per-expert counts of the stored ids for the routing that follows
 // (tk_gating_fused_topk_route); a null table when nothing is counted.
 tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int64_t H, int64_t E, int32_t k,
                             float* scores, int32_t* ids, float* logits, cudaStream_t stream,
-                            const tkg::RouteCounts& route = tkg::RouteCounts{nullptr, 0u, 0}) {
+                            const tkg::RouteCounts& route = tkg::RouteCounts{nullptr, 0u, 0},
+                            const Workspace* ws = nullptr) {
   tk_status st = validate_sizes(T, H, E, k);
   if (st != TK_OK) return st;
   if (T == 0) return TK_OK;
@@ -299,7 +353,7 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   if (dev == nullptr) return TK_ERR_CUDA;
   if (dev->status != TK_OK) return dev->status;
   tk_gating_plan pl;
-  st = plan_impl(T, H, E, k, dev->num_sms, dev->capacity, &pl);
+  st = plan_for_call(T, H, E, k, dev, ws, &pl);
   if (st != TK_OK) return st;
 
   CUtensorMap mx, mx64, mw;
@@ -311,7 +365,8 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
     return TK_ERR_CUDA;
   const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
-                           dev->clock, route};
+                           dev->clock, route, ws != nullptr ? ws->ptr : nullptr,
+                           pl.num_split_tiles > 0 ? next_split_token() : 0u};
   return tkg::launch_planned<false>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, logits, stream);
 }
 
@@ -324,7 +379,7 @@ tk_status validate_sizes_fp8(int64_t T, int64_t H, int64_t E, int32_t k) {
 
 tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale, const void* gate_q,
                                 const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k, float* scores,
-                                int32_t* ids, float* logits, cudaStream_t stream) {
+                                int32_t* ids, float* logits, cudaStream_t stream, const Workspace* ws = nullptr) {
   tk_status st = validate_sizes_fp8(T, H, E, k);
   if (st != TK_OK) return st;
   if (T == 0) return TK_OK;
@@ -337,7 +392,7 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
   if (dev->status != TK_OK) return dev->status;
   // a K slice of 128 FP8 values occupies what 64 bf16 values do: plan on H / 2
   tk_gating_plan pl;
-  st = plan_impl(T, H / 2, E, k, dev->num_sms, dev->capacity, &pl);
+  st = plan_for_call(T, H / 2, E, k, dev, ws, &pl);
   if (st != TK_OK) return st;
 
   CUtensorMap mx, mx64, mw;
@@ -349,7 +404,8 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
       !encode_2d_u8(&mw, gate_q, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kslice, tkg::B_BOX_N))
     return TK_ERR_CUDA;
   const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
-                           dev->clock, tkg::RouteCounts{nullptr, 0u, 0}};
+                           dev->clock, tkg::RouteCounts{nullptr, 0u, 0}, ws != nullptr ? ws->ptr : nullptr,
+                           pl.num_split_tiles > 0 ? next_split_token() : 0u};
   return tkg::launch_planned<true>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, logits,
                                    stream);
 }
@@ -375,6 +431,56 @@ extern "C" {
 tk_status tk_gating_fused_topk(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,
                                int32_t k, float* scores, int32_t* ids, void* stream) {
   return fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+tk_status tk_gating_fused_topk_ws(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,
+                                  int32_t k, float* scores, int32_t* ids, void* workspace, int64_t workspace_bytes,
+                                  void* stream) {
+  if (workspace_bytes < 0) return TK_ERR_INVALID_ARG;
+  const Workspace ws{workspace, workspace_bytes};
+  return fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, nullptr, static_cast<cudaStream_t>(stream),
+                           tkg::RouteCounts{nullptr, 0u, 0}, &ws);
+}
+
+tk_status tk_gating_fused_topk_ws_logits(const void* hidden, const void* gate_weight, int64_t T, int64_t H,
+                                         int64_t E, int32_t k, float* scores, int32_t* ids, float* logits,
+                                         void* workspace, int64_t workspace_bytes, void* stream) {
+  const tk_status st = validate_sizes(T, H, E, k);
+  if (st != TK_OK || T == 0) return st;
+  if (logits == nullptr || workspace_bytes < 0) return TK_ERR_INVALID_ARG;
+  if (!aligned16(logits)) return TK_ERR_ALIGNMENT;
+  const Workspace ws{workspace, workspace_bytes};
+  return fused_topk_device(hidden, gate_weight, T, H, E, k, scores, ids, logits, static_cast<cudaStream_t>(stream),
+                           tkg::RouteCounts{nullptr, 0u, 0}, &ws);
+}
+
+tk_status tk_gating_fused_topk_fp8_ws(const void* hidden_q, const float* hidden_scale, const void* gate_q,
+                                      const float* gate_scale, int64_t T, int64_t H, int64_t E, int32_t k,
+                                      float* scores, int32_t* ids, void* workspace, int64_t workspace_bytes,
+                                      void* stream) {
+  if (workspace_bytes < 0) return TK_ERR_INVALID_ARG;
+  const Workspace ws{workspace, workspace_bytes};
+  return fused_topk_fp8_device(hidden_q, hidden_scale, gate_q, gate_scale, T, H, E, k, scores, ids, nullptr,
+                               static_cast<cudaStream_t>(stream), &ws);
+}
+
+tk_status tk_gating_make_plan_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan,
+                                 int64_t* workspace_bytes) {
+  if (num_sms < 1 || plan == nullptr) return TK_ERR_INVALID_ARG;
+  return plan_impl_ws(T, H, E, k, num_sms, b200_like_capacity(num_sms), plan, workspace_bytes);
+}
+
+tk_status tk_gating_workspace_bytes(int64_t T, int64_t H, int64_t E, int32_t k, int32_t fp8,
+                                    int64_t* workspace_bytes) {
+  if (workspace_bytes == nullptr) return TK_ERR_INVALID_ARG;
+  *workspace_bytes = 0;
+  const tk_status st = fp8 ? validate_sizes_fp8(T, H, E, k) : validate_sizes(T, H, E, k);
+  if (st != TK_OK) return st;
+  const DeviceState* dev = device_state();
+  if (dev == nullptr) return TK_ERR_CUDA;
+  if (dev->status != TK_OK) return dev->status;
+  tk_gating_plan pl;
+  return plan_impl_ws(T, fp8 ? H / 2 : H, E, k, dev->num_sms, dev->capacity, &pl, workspace_bytes);
 }
 
 tk_status tk_gating_fused_topk_logits(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,

@@ -276,3 +276,50 @@ def test_fused_route_workspace_is_the_table_and_a_counter(T, k, E):
         assert p["fused_workspace_bytes"] == p["workspace_bytes"] + 16 == p["ctas"] * ((E + 3) // 4 * 4) * 4 + 16
         # a gating row's k <= 32 assignments cross at most one routing range boundary
         assert p["warp_slots"] * 32 >= 4096 >= k
+
+
+@pytest.mark.parametrize("T,H,E,k", [(65536, 7168, 256, 8), (20000, 7168, 256, 8), (65533, 4096, 200, 6),
+                                     (23000, 4096, 136, 1), (65536, 7168, 256, 4)])
+def test_workspace_plan_splits_the_last_round(T, H, E, k):
+    plain = tk.make_plan(T, H, E, k, 148)
+    plan, nbytes = tk.make_plan_ws(T, H, E, k, 148)
+    assert plain["num_half_tiles"] > 0 and plan["num_half_tiles"] == 0
+    n = plan["num_split_tiles"]
+    assert n == (plain["num_half_tiles"] + 1) // 2 and 2 * n <= plan["grid"] // 2
+    # every row is covered once: full tiles, then the split tiles (the last may run past T)
+    assert plan["num_tiles"] * 256 < T <= (plan["num_tiles"] + n) * 256
+    kb = plan["split_k_block"]
+    assert kb % 2 == 0 and 0 < kb < plan["k_blocks"]
+    cols = (E + 31) // 32 * 32
+    assert nbytes == (n * 8 + 255) // 256 * 256 + n * 256 * (cols + 4) * 4
+    # the first half's 128 rows of a CTA fit its ring once the ring is idle
+    ring = plan["smem_bytes"] - 1280
+    assert 128 * (cols + 4) * 4 <= ring
+    for key in ("variant", "block_m", "n_pad", "k_blocks", "stages", "grid", "cluster", "threads", "smem_bytes"):
+        assert plan[key] == plain[key], key
+
+
+@pytest.mark.parametrize("T,H,E,k", [(4096, 7168, 256, 8), (65536, 2048, 256, 8), (65536, 7168, 512, 8),
+                                     (60000, 4096, 256, 16), (16384, 4096, 64, 6), (1, 7168, 256, 8)])
+def test_workspace_plan_elsewhere_is_the_plain_plan(T, H, E, k):
+    assert tk.make_plan_ws(T, H, E, k, 148) == (tk.make_plan(T, H, E, k, 148), 0)
+
+
+def test_workspace_entry_points_reject_before_cuda():
+    f = tk.fused_topk_gating_ws_ptr
+    assert f(16, 16, 8, 64, 16, 17, 16, 16, 16, 1 << 20) == tk.TK_ERR_INVALID_ARG   # k > E
+    assert f(16, 16, 8, 60, 16, 2, 16, 16, 16, 1 << 20) == tk.TK_ERR_UNSUPPORTED    # H % 8
+    assert f(16, 16, 8, 64, 16, 2, 16, 16, 16, -1) == tk.TK_ERR_INVALID_ARG         # negative size
+    assert f(0, 16, 8, 64, 16, 2, 16, 16, 16, 1 << 20) == tk.TK_ERR_INVALID_ARG     # null hidden
+    assert f(16, 16, 8, 64, 16, 2, 20, 16, 16, 1 << 20) == tk.TK_ERR_ALIGNMENT      # scores
+    assert f(0, 0, 0, 64, 16, 2, 0, 0, 0, 0) == tk.TK_OK                             # T == 0
+    # valid arguments without a GPU: no CPU fallback
+    assert f(16, 16, 65536, 7168, 256, 8, 16, 16, 16, 1 << 24) in (tk.TK_ERR_CUDA, tk.TK_ERR_UNSUPPORTED)
+    lib = tk.library()
+    n = ctypes.c_int64(-1)
+    assert lib.tk_gating_workspace_bytes(8, 7168, 256, 8, 0, None) == tk.TK_ERR_INVALID_ARG
+    assert lib.tk_gating_workspace_bytes(8, 60, 256, 8, 0, ctypes.byref(n)) == tk.TK_ERR_UNSUPPORTED
+    assert lib.tk_gating_workspace_bytes(8, 7168, 256, 8, 1, ctypes.byref(n)) in (tk.TK_ERR_CUDA,
+                                                                                   tk.TK_ERR_UNSUPPORTED)
+    assert lib.tk_gating_fused_topk_fp8_ws(16, 16, 16, 16, 8, 72, 16, 2, 16, 16, 16, 1 << 20, None) == \
+        tk.TK_ERR_UNSUPPORTED                                                          # FP8: H % 16 != 0
