@@ -215,7 +215,8 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
  * The operation, outputs and errors are those of tk_gating_fused_topk
  * (section 4.1, "MoE Gating"); only the schedule of the last round differs.
  * Where the plan without workspace ends with a round of 128-token "half" tiles
- * on CTA pairs (many tokens, 64 < E <= 512, k <= 8), this call instead cuts
+ * on CTA pairs (many tokens, 64 < E <= 256, k <= 8, and long tiles: at least
+ * 96 K slices, i.e. H >= 6144 bf16 or H >= 12288 FP8 values), this call instead cuts
  * each of the last round's 256-token tiles in H between two CTA pairs: the
  * first accumulates H slices [0, split_k_block) of the tile and stores its
  * fp32 accumulator rows to the workspace, the second accumulates the rest,
@@ -228,7 +229,7 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
  *
  *   workspace        device, 16-byte aligned, at least the bytes that
  *                    tk_gating_workspace_bytes (or tk_gating_make_plan_ws)
- *                    gives for this call (8.9 MB at T = 65536, E = 256,
+ *                    gives for this call (9.1 MB at T = 65536, E = 256,
  *                    k = 8 on a B200); may be NULL when that is 0.  It starts
  *                    with flags (8 bytes per split tile, rounded up to 256)
  *                    that must be zero before the first call: zero the

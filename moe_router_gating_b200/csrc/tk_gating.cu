@@ -189,10 +189,12 @@ tk_status plan_impl_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_s
   *workspace_bytes = 0;
   const tk_status st = plan_impl(T, H, E, k, num_sms, cap, plan);
   if (st != TK_OK) return st;
-  // measured: the split pays where the tiles are long (H >= 4096) and the first
-  // half's 128 KB per CTA fits the idle ring (E <= 256)
+  // measured (65536 tokens, E = 256, k = 8; split vs plain): H = 7168 -1.7 to
+  // -2.0%, H = 4096 -0.7 to +1.6%, H = 3072 +5.5%, H = 2048 +11%, FP8 H = 7168
+  // (56 slices) +4.6 to +13%: the split pays only for long tiles, so it needs 96
+  // or more K slices, and E <= 256 (the first half's rows fit the idle ring)
   if (plan->variant != TK_VARIANT_ROW_PAIRS || plan->expert_groups != 1 || k > 8 || plan->num_half_tiles == 0 ||
-      plan->k_blocks < 64 || E > 256)
+      plan->k_blocks < 96 || E > 256)
     return TK_OK;
   const int split = (plan->num_half_tiles + 1) / 2;  // 256-token tiles; at most half the pairs take one each
   if (2 * split > plan->grid / 2) return TK_OK;

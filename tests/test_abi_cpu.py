@@ -278,8 +278,8 @@ def test_fused_route_workspace_is_the_table_and_a_counter(T, k, E):
         assert p["warp_slots"] * 32 >= 4096 >= k
 
 
-@pytest.mark.parametrize("T,H,E,k", [(65536, 7168, 256, 8), (20000, 7168, 256, 8), (65533, 4096, 200, 6),
-                                     (23000, 4096, 136, 1), (65536, 7168, 256, 4)])
+@pytest.mark.parametrize("T,H,E,k", [(65536, 7168, 256, 8), (20000, 7168, 256, 8), (65533, 6144, 200, 6),
+                                     (23000, 6144, 136, 1), (65536, 7168, 256, 4)])
 def test_workspace_plan_splits_the_last_round(T, H, E, k):
     plain = tk.make_plan(T, H, E, k, 148)
     plan, nbytes = tk.make_plan_ws(T, H, E, k, 148)
@@ -299,7 +299,7 @@ def test_workspace_plan_splits_the_last_round(T, H, E, k):
         assert plan[key] == plain[key], key
 
 
-@pytest.mark.parametrize("T,H,E,k", [(4096, 7168, 256, 8), (65536, 2048, 256, 8), (65536, 7168, 512, 8),
+@pytest.mark.parametrize("T,H,E,k", [(4096, 7168, 256, 8), (65536, 4096, 256, 8), (65536, 7168, 512, 8),
                                      (60000, 4096, 256, 16), (16384, 4096, 64, 6), (1, 7168, 256, 8)])
 def test_workspace_plan_elsewhere_is_the_plain_plan(T, H, E, k):
     assert tk.make_plan_ws(T, H, E, k, 148) == (tk.make_plan(T, H, E, k, 148), 0)

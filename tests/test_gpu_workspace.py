@@ -72,8 +72,8 @@ def run_ws(x_bits, w_bits, k, logits=False):
 @pytest.mark.parametrize("T,H,E,k", [
     (65536, 7168, 256, 8),   # the train shape: 34 split tiles
     (20000, 7168, 256, 8),   # one full round, 5 split tiles
-    (65533, 4096, 200, 6),   # ragged: the last split tile's second CTA holds rows past T
-    (23000, 4096, 136, 1),   # k = 1, E padded inside the pair halves
+    (65533, 6144, 200, 6),   # ragged: the last split tile's second CTA holds rows past T
+    (23000, 6144, 136, 1),   # k = 1, E padded inside the pair halves
 ])
 def test_split_last_round_matches_oracle(T, H, E, k):
     first, n_split, nbytes = split_rows(T, H, E, k)
@@ -174,8 +174,8 @@ def test_without_a_split_the_call_is_the_plain_one(T, H, E, k):
 
 
 def test_fp8_split_last_round_matches_fp8_oracle():
-    # FP8 slices hold 128 values of H: H = 8192 gives the 64 slices the split needs
-    T, H, E, k = 65536, 8192, 256, 8
+    # FP8 slices hold 128 values of H: H = 12288 gives the 96 slices the split needs
+    T, H, E, k = 20000, 12288, 256, 8
     wl = workloads.RouterWorkload("split_fp8", T, H, E, k, seed=9)
     assert tk.make_plan_ws(T, H // 2, E, k, _sms())[0]["num_split_tiles"] > 0
     xq, xs, wq, wsc = workloads.fp8_inputs(wl)
