@@ -638,13 +638,14 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
           continue;
         }
         if (w.split == 2) {
-          // Second H half: wait until the first half's pair has stored the same
-          // rows (one thread polls, bounded; the warps agree on the outcome)
-          // This CTA's 128 rows of the first half are contiguous in the workspace:
-          // one bulk copy brings them into the idle ring (this is the CTA's last
-          // item), where each thread then reads its row.
+          // Second H half: one thread waits (bounded) until the first half's pair
+          // has stored the same rows, then brings this CTA's 128 of them --
+          // contiguous in the workspace -- into the idle ring (this is the CTA's
+          // last item) with one bulk copy; the warps agree on the outcome, and
+          // each thread then reads its row there.
           const uint32_t rows_bytes = static_cast<uint32_t>(BLOCK_M * p.part_stride * 4);
           bool got = true;
+          bool issued = false;
           if (warp == 2 && lane == 0) {
             got = wait_split_flag(p.split_flags + 2 * w.sidx + rank, p.split_token, abort_flag, p.timeout_ns,
                                   p.err_word);
@@ -652,10 +653,12 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
             if (got && TK_CHECK(rows_bytes <= static_cast<uint32_t>(p.stages * KB_PER_STAGE *
                                                                     (A_STAGE_BYTES + p.b_boxes * B_BOX_BYTES)),
                                 p.err_word)) {
+              fence_proxy_async_global();  // the flag was acquired by ordinary loads; the copy reads asynchronously
               mbar_arrive_expect_tx(split_bar, rows_bytes);
               bulk_load_g2s(sA,
                             p.split_part + (static_cast<int64_t>(w.sidx) * (2 * BLOCK_M) + rank * BLOCK_M) * p.part_stride,
                             rows_bytes, split_bar);
+              issued = true;
             } else {
               got = false;
             }
@@ -664,6 +667,8 @@ __global__ void __launch_bounds__(row_tile_threads(KMAX, EG), 1)
           if (got) {
             got = mbar_wait(split_bar, 0, abort_flag, p.timeout_ns, ERR_WAIT_EPILOGUE, p.err_word);
             got = named_barrier_and(4, NUM_EPI_WARPS * 32, got);
+            // a copy still in flight after an expired wait lands before the CTA may exit
+            if (!got && issued) mbar_wait(split_bar, 0, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
           }
           if (got) first_half = reinterpret_cast<const float*>(sA) + (quad * 32 + lane) * p.part_stride;
         }

@@ -182,6 +182,12 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Orders this thread's view of global memory written through ordinary stores
+// (and acquired, e.g. by a flag) before its later bulk-copy reads of it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Plain (untiled) bulk copy of `bytes` contiguous bytes from global memory into
 // this CTA's shared memory, completing on `bar`; both addresses 16-byte aligned,
 // `bytes` a multiple of 16.
