@@ -172,7 +172,9 @@ typedef enum {
   TK_VARIANT_NONE = 0,        /* T == 0: nothing to launch */
   TK_VARIANT_ROW_TILES = 1,   /* persistent: each CTA owns whole 128-token tiles */
   TK_VARIANT_SPLIT_H = 2,     /* a cluster of CTAs splits H for one tile, DSMEM reduction */
-  TK_VARIANT_ROW_PAIRS = 3    /* persistent CTA pairs (tcgen05 cta_group::2), 256-token tiles */
+  TK_VARIANT_ROW_PAIRS = 3,   /* persistent CTA pairs (tcgen05 cta_group::2), 256-token tiles */
+  TK_VARIANT_FEW_TOKENS = 4   /* workspace entry points, T <= 8: CUDA-core blocks of H x 32 experts,
+                                 partial logits combined by the CTA that finishes last */
 } tk_variant;
 
 /* The launch the library makes for a problem (host logic, no GPU needed). */
@@ -196,6 +198,8 @@ typedef struct {
   int32_t num_split_tiles; /* workspace entry points: last-round 256-token tiles each split in H between two
                               CTA pairs, in place of the half tiles (0: none) */
   int32_t split_k_block;   /* the K slice (of 64) at which a split tile's H range is cut */
+  int32_t h_rows;          /* TK_VARIANT_FEW_TOKENS: rows of H per CTA (split_h CTAs per block of 32
+                              experts, n_pad / 32 blocks; block_m = T) */
 } tk_gating_plan;
 
 /*
@@ -210,11 +214,24 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
 
 /*
  * tk_gating_fused_topk_ws -- tk_gating_fused_topk with a caller-owned device
- * workspace, which lets the many-token launch end its last round sooner.
+ * workspace, which lets a call of a few tokens spread over every SM and a
+ * many-token launch end its last round sooner.
  *
  * The operation, outputs and errors are those of tk_gating_fused_topk
- * (section 4.1, "MoE Gating"); only the schedule of the last round differs.
- * Where the plan without workspace ends with a round of 128-token "half" tiles
+ * (section 4.1, "MoE Gating"); only the schedule differs, in two cases.
+ *
+ * 1 <= T <= 8 and E <= 256 (decode; plan variant TK_VARIANT_FEW_TOKENS): the
+ * launch runs about one CTA per SM, each owning a block of 32 experts and a
+ * range of H rows.  A CTA accumulates its block's partial logits on the CUDA
+ * cores (fp32, each bf16 product exact) and stores them to the workspace; the
+ * CTA that finishes last adds the partials of every logit in the order of the
+ * H ranges, selects, applies the softmax and stores.  No CTA waits for
+ * another.  The logits are fp32 sums in another association than the plain
+ * call's, so selections agree wherever the k-th and (k+1)-th logits are not
+ * within fp32 rounding.  bf16 only (the FP8 entry point keeps its plain plan
+ * for these T).
+ *
+ * Many tokens: where the plan without workspace ends with a round of 128-token "half" tiles
  * on CTA pairs (many tokens, 64 < E <= 256, k <= 8, and long tiles: at least
  * 96 K slices, i.e. H >= 6144 bf16 or H >= 12288 FP8 values), this call instead cuts
  * each of the last round's 256-token tiles in H between two CTA pairs: the
@@ -230,15 +247,17 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
  *   workspace        device, 16-byte aligned, at least the bytes that
  *                    tk_gating_workspace_bytes (or tk_gating_make_plan_ws)
  *                    gives for this call (9.1 MB at T = 65536, E = 256,
- *                    k = 8 on a B200); may be NULL when that is 0.  It starts
- *                    with flags (8 bytes per split tile, rounded up to 256)
- *                    that must be zero before the first call: zero the
- *                    workspace once after allocating it; every
- *                    call leaves them zero, so calls in order on one stream
- *                    may share a workspace.  Calls that may run at the same
- *                    time need workspaces of their own.  After a call that
- *                    reported an expired wait (tk_gating_device_error), zero
- *                    it again.
+ *                    k = 8; 147.7 KB at T = 8, H = 7168, E = 256; on a
+ *                    B200); may be NULL when that is 0.  It starts with
+ *                    flags (8 bytes per split tile, rounded up to 256) or a
+ *                    counter (the few-token case, 256 bytes) that must be
+ *                    zero before the first call: zero the workspace once
+ *                    after allocating it; every call leaves them zero, so
+ *                    calls in order on one stream may share a workspace
+ *                    whatever their sizes (one large enough for each).  Calls
+ *                    that may run at the same time need workspaces of their
+ *                    own.  After a call that reported an expired wait
+ *                    (tk_gating_device_error), zero it again.
  *   workspace_bytes  its size.
  *   the other arguments as tk_gating_fused_topk.
  *
@@ -275,11 +294,14 @@ TK_API tk_status tk_gating_fused_topk_ws_logits(const void* hidden, const void* 
 /*
  * tk_gating_make_plan_ws -- the launch tk_gating_fused_topk_ws makes for
  * (T, H, E, k) on a device like tk_gating_make_plan's, and the workspace bytes
- * it needs (0 when the launch is the one without workspace).  For the FP8
- * entry point pass H / 2.  Makes no CUDA call.
+ * it needs (0 when the launch is the one without workspace).  Makes no CUDA
+ * call.  tk_gating_make_plan_fp8_ws: the same for tk_gating_fused_topk_fp8_ws
+ * (H counts FP8 values; validated like that call).
  */
 TK_API tk_status tk_gating_make_plan_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
                                         tk_gating_plan* plan, int64_t* workspace_bytes);
+TK_API tk_status tk_gating_make_plan_fp8_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
+                                            tk_gating_plan* plan, int64_t* workspace_bytes);
 
 /*
  * tk_gating_workspace_bytes -- the workspace bytes tk_gating_fused_topk_ws

@@ -35,7 +35,7 @@ class _Plan(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in (
         "variant", "block_m", "n_pad", "num_tiles", "k_blocks", "split_h", "stages", "grid", "cluster",
         "threads", "smem_bytes", "tmem_cols", "num_half_tiles", "slices_per_stage", "expert_groups",
-        "num_split_tiles", "split_k_block")]
+        "num_split_tiles", "split_k_block", "h_rows")]
 
 
 class _RoutePlan(ctypes.Structure):
@@ -76,6 +76,8 @@ def library() -> ctypes.CDLL:
             lib.tk_gating_make_plan_ws.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(_Plan),
                                                    ctypes.POINTER(ctypes.c_int64)]
             lib.tk_gating_make_plan_ws.restype = ctypes.c_int
+            lib.tk_gating_make_plan_fp8_ws.argtypes = lib.tk_gating_make_plan_ws.argtypes
+            lib.tk_gating_make_plan_fp8_ws.restype = ctypes.c_int
             lib.tk_gating_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_int64)]
             lib.tk_gating_workspace_bytes.restype = ctypes.c_int
             lib.tk_gating_fused_topk_logits.argtypes = [vp, vp, i64, i64, i64, i32, vp, vp, vp, vp]
@@ -160,12 +162,14 @@ def gating_workspace(T: int, H: int, E: int, k: int, device=None, fp8: bool = Fa
     return torch.zeros(max(256, n), dtype=torch.uint8, device=dev)
 
 
-def make_plan_ws(T: int, H: int, E: int, k: int, num_sms: int = 148) -> tuple[dict, int]:
-    """The launch of the workspace entry point and its workspace bytes (host logic only)."""
+def make_plan_ws(T: int, H: int, E: int, k: int, num_sms: int = 148, fp8: bool = False) -> tuple[dict, int]:
+    """The launch of the workspace entry point (fp8: of the FP8 one, H in FP8 values) and its
+    workspace bytes (host logic only)."""
     p = _Plan()
     n = ctypes.c_int64(0)
-    _check(library().tk_gating_make_plan_ws(T, H, E, k, num_sms, ctypes.byref(p), ctypes.byref(n)),
-           "tk_gating_make_plan_ws")
+    fn = library().tk_gating_make_plan_fp8_ws if fp8 else library().tk_gating_make_plan_ws
+    _check(fn(T, H, E, k, num_sms, ctypes.byref(p), ctypes.byref(n)),
+           "tk_gating_make_plan_fp8_ws" if fp8 else "tk_gating_make_plan_ws")
     return {name: getattr(p, name) for name, _ in _Plan._fields_}, int(n.value)
 
 

@@ -50,8 +50,8 @@ def _inputs() -> list[str]:
 
 # Sources that compile into the fused gating kernels (not the routing kernels).
 GATING_KERNEL_SOURCES = ("tk_gating.cu", "gating_launch.cuh", "gating_launch_impl.cuh", "gating_bf16.cu",
-                         "gating_fp8.cu", "gating_row_tiles.cuh", "gating_split_h.cuh", "sm100_ptx.cuh", "route_counts.cuh",
-                         "topk_epilogue.cuh", "topk_merge.cuh")
+                         "gating_fp8.cu", "gating_row_tiles.cuh", "gating_split_h.cuh", "gating_few_tokens.cuh",
+                         "sm100_ptx.cuh", "route_counts.cuh", "topk_epilogue.cuh", "topk_merge.cuh")
 
 
 def _code_only(text: str) -> str:

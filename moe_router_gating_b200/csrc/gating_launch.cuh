@@ -11,6 +11,7 @@
 #include "tk_gating.h"
 #include "gating_row_tiles.cuh"
 #include "gating_split_h.cuh"
+#include "gating_few_tokens.cuh"
 
 namespace tkg {
 
@@ -29,9 +30,19 @@ struct LaunchEnv {
   uint64_t timeout_ns;    // bounded-wait limit
   uint64_t* clock;        // SM-clock counters of the launches (cycles, ns, launches)
   RouteCounts route;      // per-expert counts of the stored ids by routing range; table null: none
-  void* workspace;        // split last round (plan.num_split_tiles > 0): flags, then first-half partials
+  void* workspace;        // split last round (plan.num_split_tiles > 0): flags, then first-half partials;
+                          // few-token variant: its counter, then the CTAs' partial logits
   uint32_t split_token;   // non-zero, different for every launch
+  const void* hidden;     // the inputs themselves: the few-token kernel reads them with plain loads
+  const void* gate;
 };
+
+// Workspace of the few-token variant: the arrival counter (then padding to 256
+// bytes) and the CTAs' partial logits, h_blocks x T rows of n_pad floats.
+constexpr int64_t FEW_COUNTER_BYTES = 256;
+inline int64_t few_token_workspace_bytes(int64_t T, int h_blocks, int e_pad) {
+  return FEW_COUNTER_BYTES + static_cast<int64_t>(h_blocks) * T * e_pad * 4;
+}
 
 // Workspace of a split last round: num_split x 2 uint32 flags (8 bytes per tile,
 // rounded up to 256), then the first halves' fp32 rows, num_split x 256 rows of

@@ -23,6 +23,7 @@ bool set_up_kernels_of() {
             set_smem_limit(gating_split_h_kernel<KMAX, 4, FP8>) &&
             set_smem_limit(gating_split_h_kernel<KMAX, 8, FP8>) &&
             set_smem_limit(gating_split_h_kernel<KMAX, 16, FP8>);
+  if constexpr (!FP8) ok = ok && set_smem_limit(gating_few_tokens_kernel<KMAX>);
   return ok && cudaFuncSetAttribute(gating_split_h_kernel<KMAX, 16, FP8>,
                                     cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
 }
@@ -93,6 +94,22 @@ tk_status launch_split_h(const tk_gating_plan& plan, int max_cluster, const CUte
   }
 }
 
+template <int KMAX>
+tk_status launch_few_tokens(const tk_gating_plan& pl, const FewTokenParams& prm, cudaStream_t stream) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // as launch_row_tiles
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(FEW_THREADS);
+  cfg.dynamicSmemBytes = pl.smem_bytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gating_few_tokens_kernel<KMAX>, prm) != cudaSuccess) return TK_ERR_CUDA;
+  return TK_OK;
+}
+
 template <int KMAX, bool FP8>
 tk_status launch_row_variant(const tk_gating_plan& pl, const CUtensorMap& mx, const CUtensorMap& mx64,
                              const CUtensorMap& mw, const RowTileParams& prm, cudaStream_t stream) {
@@ -116,6 +133,36 @@ tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const C
                          float* scores, int32_t* ids, const float* hscale, const float* gscale, float* logits,
                          cudaStream_t stream) {
   uint32_t* err = env.err_word;
+  if (pl.variant == TK_VARIANT_FEW_TOKENS) {
+    if constexpr (FP8) {
+      return TK_ERR_UNSUPPORTED;  // the planner chooses it for bf16 inputs only
+    } else {
+      if (env.workspace == nullptr || env.hidden == nullptr || env.gate == nullptr) return TK_ERR_INVALID_ARG;
+      FewTokenParams fp;
+      fp.hidden = static_cast<const uint16_t*>(env.hidden);
+      fp.gate = static_cast<const uint16_t*>(env.gate);
+      fp.T = static_cast<int32_t>(T);
+      fp.H = static_cast<int32_t>(H);
+      fp.E = static_cast<int32_t>(E);
+      fp.k = k;
+      fp.e_blocks = pl.n_pad / FEW_EXPERTS;
+      fp.h_blocks = pl.split_h;
+      fp.h_rows = pl.h_rows;
+      fp.e_pad = pl.n_pad;
+      fp.counter = static_cast<uint32_t*>(env.workspace);
+      fp.part = reinterpret_cast<float*>(static_cast<uint8_t*>(env.workspace) + FEW_COUNTER_BYTES);
+      fp.scores = scores;
+      fp.ids = ids;
+      fp.logits = logits;
+      fp.err_word = err;
+      fp.timeout_ns = env.timeout_ns;
+      fp.clock = env.clock;
+      if (k <= 4) return launch_few_tokens<4>(pl, fp, stream);
+      if (k <= 8) return launch_few_tokens<8>(pl, fp, stream);
+      if (k <= 16) return launch_few_tokens<16>(pl, fp, stream);
+      return launch_few_tokens<32>(pl, fp, stream);
+    }
+  }
   if (pl.variant == TK_VARIANT_SPLIT_H) {
     SplitHParams sp;
     sp.T = static_cast<int32_t>(T);

@@ -178,17 +178,60 @@ tk_status plan_impl(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
   return TK_OK;
 }
 
+// Few-token plan (bf16, T <= FEW_MAX_TOKENS): ceil(E / 32) blocks of 32 experts,
+// each split in H over h_blocks CTAs of h_rows rows (a multiple of 8), about one
+// CTA per SM in all.  TK_ERR_UNSUPPORTED when its shared memory does not fit.
+tk_status plan_few_tokens(int64_t T, int64_t H, int64_t E, int32_t num_sms, tk_gating_plan* plan,
+                          int64_t* workspace_bytes) {
+  const int e_blocks = static_cast<int>((E + tkg::FEW_EXPERTS - 1) / tkg::FEW_EXPERTS);
+  int64_t h_blocks = std::max<int64_t>(1, num_sms / e_blocks);
+  h_blocks = std::min<int64_t>(h_blocks, H / 8);
+  const int64_t h_rows = (H + h_blocks - 1) / h_blocks;
+  const int h_rows8 = static_cast<int>((h_rows + 7) / 8 * 8);
+  h_blocks = (H + h_rows8 - 1) / h_rows8;  // no empty block
+  const int e_pad = e_blocks * tkg::FEW_EXPERTS;
+  const tkg::FewTokenSmem lay = tkg::few_token_smem(static_cast<int>(T), h_rows8, static_cast<int>(h_blocks), e_pad);
+  if (lay.total > kMaxDynamicSmem) return TK_ERR_UNSUPPORTED;
+  std::memset(plan, 0, sizeof(*plan));
+  plan->variant = TK_VARIANT_FEW_TOKENS;
+  plan->block_m = static_cast<int32_t>(T);
+  plan->n_pad = e_pad;
+  plan->num_tiles = 1;
+  plan->k_blocks = static_cast<int32_t>((H + tkg::BLOCK_K - 1) / tkg::BLOCK_K);
+  plan->split_h = static_cast<int32_t>(h_blocks);
+  plan->grid = static_cast<int32_t>(h_blocks * e_blocks);
+  plan->cluster = 1;
+  plan->threads = tkg::FEW_THREADS;
+  plan->smem_bytes = lay.total;
+  plan->expert_groups = 1;
+  plan->h_rows = h_rows8;
+  *workspace_bytes = tkg::few_token_workspace_bytes(T, static_cast<int>(h_blocks), e_pad);
+  return TK_OK;
+}
+
 // The plan of the workspace entry points (tk_gating_fused_topk_ws): the plan
-// without workspace, except that a last round of half tiles on CTA pairs (one
-// expert group, lists of at most 8) becomes ceil(half tiles / 2) 256-token tiles
-// each split in H between two pairs; *workspace_bytes is what that needs (0 when
-// nothing is split).
+// without workspace, except that
+//  * bf16 calls of at most FEW_MAX_TOKENS tokens (E <= 256) run the few-token
+//    kernel, whose CTAs combine their partial logits through the workspace;
+//  * a last round of half tiles on CTA pairs (one expert group, lists of at
+//    most 8) becomes ceil(half tiles / 2) 256-token tiles each split in H
+//    between two pairs.
+// *workspace_bytes is what the plan needs (0 when it is the plain one).
 tk_status plan_impl_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, const ClusterCapacity& cap,
-                       tk_gating_plan* plan, int64_t* workspace_bytes) {
+                       bool fp8, tk_gating_plan* plan, int64_t* workspace_bytes) {
   if (workspace_bytes == nullptr) return TK_ERR_INVALID_ARG;
   *workspace_bytes = 0;
   const tk_status st = plan_impl(T, H, E, k, num_sms, cap, plan);
   if (st != TK_OK) return st;
+  if (!fp8 && T >= 1 && T <= tkg::FEW_MAX_TOKENS && E <= 256) {
+    tk_gating_plan few;
+    int64_t bytes = 0;
+    if (plan_few_tokens(T, H, E, num_sms, &few, &bytes) == TK_OK) {
+      *plan = few;
+      *workspace_bytes = bytes;
+      return TK_OK;
+    }
+  }
   // measured (65536 tokens, E = 256, k = 8; split vs plain): H = 7168 -1.7 to
   // -2.0%, H = 4096 -0.7 to +1.6%, H = 3072 +5.5%, H = 2048 +11%, FP8 H = 7168
   // (56 slices) +4.6 to +13%: the split pays only for long tiles, so it needs 96
@@ -330,10 +373,10 @@ uint32_t next_split_token() {
 // Plan on the current device: without a workspace, or the workspace plan, whose
 // bytes the caller's workspace must hold (checked before any launch).
 tk_status plan_for_call(int64_t T, int64_t H, int64_t E, int32_t k, const DeviceState* dev, const Workspace* ws,
-                        tk_gating_plan* pl) {
+                        bool fp8, tk_gating_plan* pl) {
   if (ws == nullptr) return plan_impl(T, H, E, k, dev->num_sms, dev->capacity, pl);
   int64_t need = 0;
-  const tk_status st = plan_impl_ws(T, H, E, k, dev->num_sms, dev->capacity, pl, &need);
+  const tk_status st = plan_impl_ws(T, H, E, k, dev->num_sms, dev->capacity, fp8, pl, &need);
   if (st != TK_OK) return st;
   if (need > 0 && (ws->ptr == nullptr || ws->bytes < need)) return TK_ERR_INVALID_ARG;
   if (need > 0 && !aligned16(ws->ptr)) return TK_ERR_ALIGNMENT;
@@ -355,20 +398,23 @@ tk_status fused_topk_device(const void* hidden, const void* gate, int64_t T, int
   if (dev == nullptr) return TK_ERR_CUDA;
   if (dev->status != TK_OK) return dev->status;
   tk_gating_plan pl;
-  st = plan_for_call(T, H, E, k, dev, ws, &pl);
+  st = plan_for_call(T, H, E, k, dev, ws, false, &pl);
   if (st != TK_OK) return st;
 
   CUtensorMap mx, mx64, mw;
+  std::memset(&mx, 0, sizeof(mx));
   std::memset(&mx64, 0, sizeof(mx64));
-  if (!encode_2d_bf16(&mx, hidden, static_cast<uint64_t>(T), static_cast<uint64_t>(H), tkg::BLOCK_K,
-                      tkg::BLOCK_M) ||
-      (pl.num_half_tiles > 0 && !encode_2d_bf16(&mx64, hidden, static_cast<uint64_t>(T), static_cast<uint64_t>(H),
-                                                tkg::BLOCK_K, tkg::BLOCK_M / 2)) ||
-      !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K))
+  std::memset(&mw, 0, sizeof(mw));
+  if (pl.variant != TK_VARIANT_FEW_TOKENS &&  // that kernel reads the inputs with plain loads
+      (!encode_2d_bf16(&mx, hidden, static_cast<uint64_t>(T), static_cast<uint64_t>(H), tkg::BLOCK_K,
+                       tkg::BLOCK_M) ||
+       (pl.num_half_tiles > 0 && !encode_2d_bf16(&mx64, hidden, static_cast<uint64_t>(T),
+                                                 static_cast<uint64_t>(H), tkg::BLOCK_K, tkg::BLOCK_M / 2)) ||
+       !encode_2d_bf16(&mw, gate, static_cast<uint64_t>(H), static_cast<uint64_t>(E), tkg::B_BOX_N, tkg::BLOCK_K)))
     return TK_ERR_CUDA;
   const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
                            dev->clock, route, ws != nullptr ? ws->ptr : nullptr,
-                           pl.num_split_tiles > 0 ? next_split_token() : 0u};
+                           pl.num_split_tiles > 0 ? next_split_token() : 0u, hidden, gate};
   return tkg::launch_planned<false>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, nullptr, nullptr, logits, stream);
 }
 
@@ -394,7 +440,7 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
   if (dev->status != TK_OK) return dev->status;
   // a K slice of 128 FP8 values occupies what 64 bf16 values do: plan on H / 2
   tk_gating_plan pl;
-  st = plan_for_call(T, H / 2, E, k, dev, ws, &pl);
+  st = plan_for_call(T, H / 2, E, k, dev, ws, true, &pl);
   if (st != TK_OK) return st;
 
   CUtensorMap mx, mx64, mw;
@@ -407,7 +453,7 @@ tk_status fused_topk_fp8_device(const void* hidden_q, const float* hidden_scale,
     return TK_ERR_CUDA;
   const tkg::LaunchEnv env{dev->max_split_cluster, dev->err_word, g_timeout_ns.load(std::memory_order_relaxed),
                            dev->clock, tkg::RouteCounts{nullptr, 0u, 0}, ws != nullptr ? ws->ptr : nullptr,
-                           pl.num_split_tiles > 0 ? next_split_token() : 0u};
+                           pl.num_split_tiles > 0 ? next_split_token() : 0u, hidden_q, gate_q};
   return tkg::launch_planned<true>(pl, env, mx, mx64, mw, T, H, E, k, scores, ids, hidden_scale, gate_scale, logits,
                                    stream);
 }
@@ -469,7 +515,19 @@ tk_status tk_gating_fused_topk_fp8_ws(const void* hidden_q, const float* hidden_
 tk_status tk_gating_make_plan_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms, tk_gating_plan* plan,
                                  int64_t* workspace_bytes) {
   if (num_sms < 1 || plan == nullptr) return TK_ERR_INVALID_ARG;
-  return plan_impl_ws(T, H, E, k, num_sms, b200_like_capacity(num_sms), plan, workspace_bytes);
+  return plan_impl_ws(T, H, E, k, num_sms, b200_like_capacity(num_sms), false, plan, workspace_bytes);
+}
+
+tk_status tk_gating_make_plan_fp8_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_sms,
+                                     tk_gating_plan* plan, int64_t* workspace_bytes) {
+  if (num_sms < 1 || plan == nullptr) return TK_ERR_INVALID_ARG;
+  const tk_status st = validate_sizes_fp8(T, H, E, k);
+  if (st != TK_OK) {
+    std::memset(plan, 0, sizeof(*plan));
+    if (workspace_bytes != nullptr) *workspace_bytes = 0;
+    return st;
+  }
+  return plan_impl_ws(T, H / 2, E, k, num_sms, b200_like_capacity(num_sms), true, plan, workspace_bytes);
 }
 
 tk_status tk_gating_workspace_bytes(int64_t T, int64_t H, int64_t E, int32_t k, int32_t fp8,
@@ -482,7 +540,7 @@ tk_status tk_gating_workspace_bytes(int64_t T, int64_t H, int64_t E, int32_t k, 
   if (dev == nullptr) return TK_ERR_CUDA;
   if (dev->status != TK_OK) return dev->status;
   tk_gating_plan pl;
-  return plan_impl_ws(T, fp8 ? H / 2 : H, E, k, dev->num_sms, dev->capacity, &pl, workspace_bytes);
+  return plan_impl_ws(T, fp8 ? H / 2 : H, E, k, dev->num_sms, dev->capacity, fp8 != 0, &pl, workspace_bytes);
 }
 
 tk_status tk_gating_fused_topk_logits(const void* hidden, const void* gate_weight, int64_t T, int64_t H, int64_t E,

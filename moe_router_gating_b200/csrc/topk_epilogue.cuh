@@ -29,18 +29,24 @@ struct RowTopK {
   // j holds the old slot j when !c_j, the old slot j-1 when c_{j-1} (the list is
   // sorted, so c_{j-1} implies c_j), and the offered pair otherwise.  All slot
   // updates read the old list, so they are independent of one another, and no
-  // lane of a warp ever waits on another lane's insertion.
+  // lane of a warp ever waits on another lane's insertion.  The comparisons are
+  // taken into one bit mask before any slot changes: written as an array of
+  // bools, nvcc 12.9 for sm_100a was seen to build lists of 4 that held the
+  // offered pair twice (the list's first comparison redone against the updated
+  // slot 0), in some loop contexts only.
   __device__ __forceinline__ void offer(float value, int32_t index) {
-    bool c[KMAX];
+    uint32_t c = 0;
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) c[j] = value > v[j];
+    for (int j = 0; j < KMAX; ++j) c |= static_cast<uint32_t>(value > v[j]) << j;
 #pragma unroll
     for (int j = KMAX - 1; j > 0; --j) {
-      v[j] = c[j] ? (c[j - 1] ? v[j - 1] : value) : v[j];
-      i[j] = c[j] ? (c[j - 1] ? i[j - 1] : index) : i[j];
+      const bool cj = (c >> j) & 1u;
+      const bool cp = (c >> (j - 1)) & 1u;
+      v[j] = cj ? (cp ? v[j - 1] : value) : v[j];
+      i[j] = cj ? (cp ? i[j - 1] : index) : i[j];
     }
-    v[0] = c[0] ? value : v[0];
-    i[0] = c[0] ? index : i[0];
+    v[0] = (c & 1u) ? value : v[0];
+    i[0] = (c & 1u) ? index : i[0];
   }
 
   // Offer a candidate whose index may be lower than ones already held (used when

@@ -300,9 +300,33 @@ def test_workspace_plan_splits_the_last_round(T, H, E, k):
 
 
 @pytest.mark.parametrize("T,H,E,k", [(4096, 7168, 256, 8), (65536, 4096, 256, 8), (65536, 7168, 512, 8),
-                                     (60000, 4096, 256, 16), (16384, 4096, 64, 6), (1, 7168, 256, 8)])
+                                     (60000, 4096, 256, 16), (16384, 4096, 64, 6), (9, 7168, 256, 8),
+                                     (1, 7168, 512, 8)])
 def test_workspace_plan_elsewhere_is_the_plain_plan(T, H, E, k):
     assert tk.make_plan_ws(T, H, E, k, 148) == (tk.make_plan(T, H, E, k, 148), 0)
+
+
+@pytest.mark.parametrize("num_sms", [148, 132, 16])
+@pytest.mark.parametrize("T,H,E,k", [(1, 7168, 256, 8), (8, 7168, 256, 8), (3, 4096, 64, 6), (8, 512, 16, 2),
+                                     (7, 2048, 200, 8), (6, 1000, 96, 16), (1, 8, 16, 4), (4, 7168, 256, 32)])
+def test_workspace_plan_few_tokens(T, H, E, k, num_sms):
+    plan, nbytes = tk.make_plan_ws(T, H, E, k, num_sms)
+    assert plan["variant"] == 4 and plan["block_m"] == T and plan["cluster"] == 1 and plan["threads"] == 256
+    e_blocks = (E + 31) // 32
+    hb, rows = plan["split_h"], plan["h_rows"]
+    assert plan["n_pad"] == 32 * e_blocks and plan["grid"] == hb * e_blocks <= max(num_sms, e_blocks)
+    # the H ranges: multiples of 8 rows, none empty, covering H once
+    assert rows % 8 == 0 and (hb - 1) * rows < H <= hb * rows
+    # the counter (256 bytes), then h_blocks x T partial rows of n_pad floats
+    assert nbytes == 256 + hb * T * plan["n_pad"] * 4
+    # shared memory: barrier and flag, staged hidden values, the warps' sums, the copied partials, the sums
+    def up(v):
+        return (v + 127) // 128 * 128
+    smem = 128 + up(T * rows * 4) + 8 * T * 32 * 4 + up(hb * T * plan["n_pad"] * 4) + T * plan["n_pad"] * 4
+    assert plan["smem_bytes"] == smem <= 232448
+    # the FP8 entry point keeps its plain plan
+    if H % 16 == 0:
+        assert tk.make_plan_ws(T, H, E, k, num_sms, fp8=True) == (tk.make_plan(T, H // 2, E, k, num_sms), 0)
 
 
 def test_workspace_entry_points_reject_before_cuda():
