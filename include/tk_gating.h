@@ -173,7 +173,7 @@ typedef enum {
   TK_VARIANT_ROW_TILES = 1,   /* persistent: each CTA owns whole 128-token tiles */
   TK_VARIANT_SPLIT_H = 2,     /* a cluster of CTAs splits H for one tile, DSMEM reduction */
   TK_VARIANT_ROW_PAIRS = 3,   /* persistent CTA pairs (tcgen05 cta_group::2), 256-token tiles */
-  TK_VARIANT_FEW_TOKENS = 4   /* workspace entry points, T <= 8: CUDA-core blocks of H x 32 experts,
+  TK_VARIANT_FEW_TOKENS = 4   /* workspace entry points, T <= 4: CUDA-core blocks of H x 32 experts,
                                  partial logits combined by the CTA that finishes last */
 } tk_variant;
 
@@ -220,7 +220,7 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
  * The operation, outputs and errors are those of tk_gating_fused_topk
  * (section 4.1, "MoE Gating"); only the schedule differs, in two cases.
  *
- * 1 <= T <= 8 and E <= 256 (decode; plan variant TK_VARIANT_FEW_TOKENS): the
+ * 1 <= T <= 4 and E <= 256 (decode; plan variant TK_VARIANT_FEW_TOKENS): the
  * launch runs about one CTA per SM, each owning a block of 32 experts and a
  * range of H rows.  A CTA accumulates its block's partial logits on the CUDA
  * cores (fp32, each bf16 product exact) and stores them to the workspace; the
@@ -247,7 +247,7 @@ TK_API tk_status tk_gating_make_plan(int64_t T, int64_t H, int64_t E, int32_t k,
  *   workspace        device, 16-byte aligned, at least the bytes that
  *                    tk_gating_workspace_bytes (or tk_gating_make_plan_ws)
  *                    gives for this call (9.1 MB at T = 65536, E = 256,
- *                    k = 8; 147.7 KB at T = 8, H = 7168, E = 256; on a
+ *                    k = 8; 74.0 KB at T = 4, H = 7168, E = 256; on a
  *                    B200); may be NULL when that is 0.  It starts with
  *                    flags (8 bytes per split tile, rounded up to 256) or a
  *                    counter (the few-token case, 256 bytes) that must be

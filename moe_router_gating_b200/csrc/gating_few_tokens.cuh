@@ -24,8 +24,9 @@
 //      merged by shuffles), applies the softmax over them and stores.
 //
 // No CTA waits for another: the last one finds every other block's partials
-// stored (each CTA fences its stores before it counts itself).  The last CTA
-// sets the counter back to zero, so it is zero between launches.
+// stored (each CTA counts itself with a release after its stores, the count
+// that finds all others there is an acquire).  The last CTA sets the counter
+// back to zero, so it is zero between launches.
 //
 // The selection and softmax are those of the other gating kernels (the naive
 // form on the chenxutan.com page "TileKernels 深度解析", section 4.1:
@@ -43,8 +44,9 @@ namespace tkg {
 
 constexpr int FEW_THREADS = 256;
 constexpr int FEW_WARPS = FEW_THREADS / 32;
-constexpr int FEW_MAX_TOKENS = 8;   // tokens per launch of this kernel
+constexpr int FEW_MAX_TOKENS = 4;   // tokens per launch of this kernel (from 4 on, split-H is as fast)
 constexpr int FEW_EXPERTS = 32;     // experts per CTA: four 16-byte slots of 8
+constexpr int FEW_MAX_EXPERTS = 256;  // E of a few-token call: at most 8 experts per lane in the selection
 constexpr int FEW_ROW_GROUPS = FEW_THREADS / 4;  // threads sharing a slot: rows r, r + 64, ...
 constexpr int FEW_BATCH = 8;        // gate rows per thread in flight
 constexpr int FEW_COPY_CHUNK = 32768;  // bytes per bulk copy of the partials
@@ -217,17 +219,18 @@ __global__ void __launch_bounds__(FEW_THREADS, 1) gating_few_tokens_kernel(const
     p.part[(static_cast<int64_t>(hb) * T + t) * p.e_pad + eb * FEW_EXPERTS + e] = s;
   }
 
-  // count this CTA done; the last one combines
-  __threadfence();
+  // count this CTA done; the last one combines.  The barrier orders every
+  // thread's partial stores before thread 0's arrival, whose release (gpu
+  // scope, cumulative) publishes them; its acquire lets the last CTA read
+  // the other CTAs' partials.
   __syncthreads();
   const uint32_t num_ctas = static_cast<uint32_t>(p.e_blocks * p.h_blocks);
   if (tid == 0) {
-    const uint32_t before = atomicAdd(p.counter, 1u);
+    const uint32_t before = atom_add_acq_rel_gpu(p.counter, 1u);
     const int last = before == num_ctas - 1;
     *last_flag = last;
     if (last) {
-      __threadfence();
-      atomicExch(p.counter, 0u);  // every CTA of this launch has counted itself
+      *p.counter = 0u;  // every CTA of this launch has counted itself
       fence_proxy_async_global();  // the partials were stored by ordinary stores; the copies read them asynchronously
       const uint32_t total = static_cast<uint32_t>(p.h_blocks * T * p.e_pad * 4);
       mbar_arrive_expect_tx(bar, total);
@@ -247,11 +250,22 @@ __global__ void __launch_bounds__(FEW_THREADS, 1) gating_few_tokens_kernel(const
     mbar_wait(bar, 0, nullptr, DRAIN_TIMEOUT_NS, ERR_WAIT_DRAIN, p.err_word);
     return;
   }
+  const int part_stride = T * p.e_pad;  // floats from one H range's partial to the next
   for (int q = tid; q < T * p.E; q += FEW_THREADS) {
     const int t = q / p.E;
     const int e = q - t * p.E;
-    float s = parts[t * p.e_pad + e];
-    for (int h = 1; h < p.h_blocks; ++h) s += parts[(h * T + t) * p.e_pad + e];
+    const float* src = parts + t * p.e_pad + e;
+    // added in the order of the H ranges; eight loads issued ahead of their additions
+    float s = src[0];
+    int h = 1;
+    for (; h + 8 <= p.h_blocks; h += 8) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = src[(h + j) * part_stride];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += v[j];
+    }
+    for (; h < p.h_blocks; ++h) s += src[h * part_stride];
     sums[t * p.e_pad + e] = s;
     if (p.logits != nullptr) p.logits[static_cast<int64_t>(t) * p.E + e] = s;
   }
@@ -265,7 +279,12 @@ __global__ void __launch_bounds__(FEW_THREADS, 1) gating_few_tokens_kernel(const
     top.reset();
     const int e_begin = lane * per_lane;
     const int e_end = min(p.E, e_begin + per_lane);
-    for (int e = e_begin; e < e_end; ++e) top.offer(sums[t * p.e_pad + e], e);
+    float v[FEW_MAX_EXPERTS / 32];  // the lane's values, loaded before its offers
+#pragma unroll
+    for (int j = 0; j < FEW_MAX_EXPERTS / 32; ++j) v[j] = e_begin + j < e_end ? sums[t * p.e_pad + e_begin + j] : 0.0f;
+#pragma unroll
+    for (int j = 0; j < FEW_MAX_EXPERTS / 32; ++j)
+      if (e_begin + j < e_end) top.offer(v[j], e_begin + j);
     merge_lane_groups(top, 32);
     group_softmax_store(top, p.k, 32, true, p.scores + static_cast<int64_t>(t) * p.k,
                         p.ids + static_cast<int64_t>(t) * p.k);

@@ -182,6 +182,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Atomic add at gpu scope with acquire-release semantics; returns the old value.
+// After a CTA barrier, one thread's release publishes the stores of every thread
+// of the CTA that came before the barrier.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
 // Orders this thread's view of global memory written through ordinary stores
 // (and acquired, e.g. by a flag) before its later bulk-copy reads of it.
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -223,7 +223,7 @@ tk_status plan_impl_ws(int64_t T, int64_t H, int64_t E, int32_t k, int32_t num_s
   *workspace_bytes = 0;
   const tk_status st = plan_impl(T, H, E, k, num_sms, cap, plan);
   if (st != TK_OK) return st;
-  if (!fp8 && T >= 1 && T <= tkg::FEW_MAX_TOKENS && E <= 256) {
+  if (!fp8 && T >= 1 && T <= tkg::FEW_MAX_TOKENS && E <= tkg::FEW_MAX_EXPERTS) {
     tk_gating_plan few;
     int64_t bytes = 0;
     if (plan_few_tokens(T, H, E, num_sms, &few, &bytes) == TK_OK) {

@@ -300,15 +300,15 @@ def test_workspace_plan_splits_the_last_round(T, H, E, k):
 
 
 @pytest.mark.parametrize("T,H,E,k", [(4096, 7168, 256, 8), (65536, 4096, 256, 8), (65536, 7168, 512, 8),
-                                     (60000, 4096, 256, 16), (16384, 4096, 64, 6), (9, 7168, 256, 8),
-                                     (1, 7168, 512, 8)])
+                                     (60000, 4096, 256, 16), (16384, 4096, 64, 6), (5, 7168, 256, 8),
+                                     (8, 7168, 256, 8), (1, 7168, 512, 8)])
 def test_workspace_plan_elsewhere_is_the_plain_plan(T, H, E, k):
     assert tk.make_plan_ws(T, H, E, k, 148) == (tk.make_plan(T, H, E, k, 148), 0)
 
 
 @pytest.mark.parametrize("num_sms", [148, 132, 16])
-@pytest.mark.parametrize("T,H,E,k", [(1, 7168, 256, 8), (8, 7168, 256, 8), (3, 4096, 64, 6), (8, 512, 16, 2),
-                                     (7, 2048, 200, 8), (6, 1000, 96, 16), (1, 8, 16, 4), (4, 7168, 256, 32)])
+@pytest.mark.parametrize("T,H,E,k", [(1, 7168, 256, 8), (4, 7168, 256, 8), (3, 4096, 64, 6), (4, 512, 16, 2),
+                                     (3, 2048, 200, 8), (2, 1000, 96, 16), (1, 8, 16, 4), (4, 7168, 256, 32)])
 def test_workspace_plan_few_tokens(T, H, E, k, num_sms):
     plan, nbytes = tk.make_plan_ws(T, H, E, k, num_sms)
     assert plan["variant"] == 4 and plan["block_m"] == T and plan["cluster"] == 1 and plan["threads"] == 256
