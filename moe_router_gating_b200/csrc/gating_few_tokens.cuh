@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(FEW_THREADS, 1) gating_few_tokens_kernel(const
     for (int q = tid; q < T * chunks; q += FEW_THREADS) {
       const int t = q / chunks;
       const int c = q - t * chunks;
+      // the token's row slice inside hidden and inside the staging area
+      if (!TK_CHECK(h0 + 8 * c + 8 <= p.H && (t * p.h_rows + 8 * c + 8) * 4 <= lay.red - lay.xs, p.err_word)) break;
       const uint4 v = ldg_nc_v4(p.hidden + static_cast<int64_t>(t) * p.H + h0 + 8 * c);
       float4* dst = reinterpret_cast<float4*>(xs + t * p.h_rows + 8 * c);
       dst[0] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(FEW_THREADS, 1) gating_few_tokens_kernel(const
     float s = red[t * FEW_EXPERTS + e];
 #pragma unroll
     for (int w = 1; w < FEW_WARPS; ++w) s += red[(w * T + t) * FEW_EXPERTS + e];
+    if (!TK_CHECK(hb < p.h_blocks && eb * FEW_EXPERTS + e < p.e_pad, p.err_word)) break;
     p.part[(static_cast<int64_t>(hb) * T + t) * p.e_pad + eb * FEW_EXPERTS + e] = s;
   }
 
@@ -232,7 +235,9 @@ __global__ void __launch_bounds__(FEW_THREADS, 1) gating_few_tokens_kernel(const
     if (last) {
       *p.counter = 0u;  // every CTA of this launch has counted itself
       fence_proxy_async_global();  // the partials were stored by ordinary stores; the copies read them asynchronously
-      const uint32_t total = static_cast<uint32_t>(p.h_blocks * T * p.e_pad * 4);
+      uint32_t total = static_cast<uint32_t>(p.h_blocks * T * p.e_pad * 4);
+      // the partials fit the shared-memory area they are copied to (else: no copy, the arrival alone)
+      if (!TK_CHECK(total <= static_cast<uint32_t>(lay.sums - lay.parts), p.err_word)) total = 0;
       mbar_arrive_expect_tx(bar, total);
       for (uint32_t off = 0; off < total; off += FEW_COPY_CHUNK) {
         const uint32_t n = total - off < static_cast<uint32_t>(FEW_COPY_CHUNK) ? total - off

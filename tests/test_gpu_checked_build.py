@@ -20,8 +20,8 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # (T, H, E, k): one CTA per tile, CTA pairs with half tiles, two MMA chunks, two
-# expert groups, split-H clusters of 16 / 4 / 8; FP8 and the workspace entry
-# point's split last round below
+# expert groups, split-H clusters of 16 / 4 / 8; FP8, the workspace entry
+# point's split last round and its few-token kernel below
 CASES = [(20000, 512, 64, 4), (20000, 512, 256, 8), (24000, 256, 512, 8), (20000, 256, 1024, 8),
          (1, 7168, 256, 8), (4096, 1024, 256, 8), (300, 520, 40, 3), (300, 256, 1024, 32)]
 
@@ -46,6 +46,10 @@ wl = workloads.RouterWorkload("chkws", 20000, 7168, 256, 8, seed=33)
 x = workloads.to_torch_bf16(wl.hidden()).cuda(); w = workloads.to_torch_bf16(wl.gate_weight()).cuda()
 sw, iw = tk.fused_topk_gating(x, w, 8, workspace=tk.gating_workspace(20000, 7168, 256, 8))
 out["split"] = [sw.cpu().numpy(), iw.cpu().numpy()]
+wl = workloads.RouterWorkload("chkfew", 3, 7168, 200, 8, seed=34)
+x = workloads.to_torch_bf16(wl.hidden()).cuda(); w = workloads.to_torch_bf16(wl.gate_weight()).cuda()
+sf, i_f = tk.fused_topk_gating(x, w, 8, workspace=tk.gating_workspace(3, 7168, 200, 8))
+out["few"] = [sf.cpu().numpy(), i_f.cpu().numpy()]
 g = ep.ExpertParallelGroup(64, 512, capacity=20000 * 4)
 xt = workloads.to_torch_bf16(workloads.normal_bf16(5, 1, 0, 20000 * 512).reshape(20000, 512)).cuda()
 ids = torch.from_numpy(workloads.expert_ids(20000, 4, 64, seed=5, kind="skew")).cuda()
@@ -85,6 +89,12 @@ def test_checked_build_runs_clean_and_matches_release(tmp_path):
     w = workloads.to_torch_bf16(wl.gate_weight()).cuda()
     sw, iw = tk.fused_topk_gating(x, w, 8, workspace=tk.gating_workspace(20000, 7168, 256, 8))
     assert np.array_equal(sw.cpu().numpy(), got["split"][0]) and np.array_equal(iw.cpu().numpy(), got["split"][1])
+    # the few-token kernel of the workspace entry point (3 tokens, E not a multiple of 32)
+    wl = workloads.RouterWorkload("chkfew", 3, 7168, 200, 8, seed=34)
+    x = workloads.to_torch_bf16(wl.hidden()).cuda()
+    w = workloads.to_torch_bf16(wl.gate_weight()).cuda()
+    sf, i_f = tk.fused_topk_gating(x, w, 8, workspace=tk.gating_workspace(3, 7168, 200, 8))
+    assert np.array_equal(sf.cpu().numpy(), got["few"][0]) and np.array_equal(i_f.cpu().numpy(), got["few"][1])
     g = ep.ExpertParallelGroup(64, 512, capacity=20000 * 4)
     xt = workloads.to_torch_bf16(workloads.normal_bf16(5, 1, 0, 20000 * 512).reshape(20000, 512)).cuda()
     ids = torch.from_numpy(workloads.expert_ids(20000, 4, 64, seed=5, kind="skew")).cuda()
