@@ -138,6 +138,7 @@ tk_status launch_planned(const tk_gating_plan& pl, const LaunchEnv& env, const C
       return TK_ERR_UNSUPPORTED;  // the planner chooses it for bf16 inputs only
     } else {
       if (env.workspace == nullptr || env.hidden == nullptr || env.gate == nullptr) return TK_ERR_INVALID_ARG;
+      if (env.route.table != nullptr) return TK_ERR_UNSUPPORTED;  // this kernel takes no routing counts
       FewTokenParams fp;
       fp.hidden = static_cast<const uint16_t*>(env.hidden);
       fp.gate = static_cast<const uint16_t*>(env.gate);

@@ -168,3 +168,25 @@ def test_decode_workloads():
 def test_fp8_keeps_its_plain_plan():
     plan, nbytes = tk.make_plan_ws(1, 7168, 256, 8, _sms(), fp8=True)
     assert plan["variant"] == 2 and nbytes == 0
+
+
+def test_right_after_a_kernel_that_writes_hidden():
+    """The few-token kernel is launched as a programmatic dependent of the previous
+    kernel: its loads (plain 16-byte loads, not TMA) must still see what that
+    kernel wrote -- here a copy into the hidden buffer just before each call."""
+    wl = workloads.RouterWorkload("few_pdl", 2, 7168, 256, 8, seed=23)
+    a_bits = wl.hidden()
+    b_bits = workloads.RouterWorkload(wl.name, wl.T, wl.H, wl.E, wl.k, seed=wl.seed + 100).hidden()
+    w_bits = wl.gate_weight()
+    a, b, w = to_device_bf16(a_bits), to_device_bf16(b_bits), to_device_bf16(w_bits)
+    x = torch.empty_like(a)
+    ws = tk.gating_workspace(wl.T, wl.H, wl.E, wl.k)
+    results = []
+    for src in (a, b, a, b):
+        x.copy_(src)
+        s, i = tk.fused_topk_gating(x, w, wl.k, workspace=ws)
+        results.append((s.clone(), i.clone()))
+    torch.cuda.synchronize()
+    for bits, (s, i) in zip((a_bits, b_bits, a_bits, b_bits), results):
+        ref = oracle.fused_topk_gating(bits, w_bits, wl.k, want_logits=True)
+        parity.check(s.cpu().numpy(), i.cpu().numpy(), ref, label=wl.name)
