@@ -190,3 +190,27 @@ def test_right_after_a_kernel_that_writes_hidden():
     for bits, (s, i) in zip((a_bits, b_bits, a_bits, b_bits), results):
         ref = oracle.fused_topk_gating(bits, w_bits, wl.k, want_logits=True)
         parity.check(s.cpu().numpy(), i.cpu().numpy(), ref, label=wl.name)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 256, 8), (4, 64, 8), (3, 200, 32), (2, 16, 16)])
+def test_zero_gate_gives_uniform_scores(T, E, k):
+    """Every logit is 0: all ties, so the ids are 0..k-1 (lower index first) and the
+    scores 1/k -- the tie order across lanes, lane merges and expert blocks."""
+    H = 2048
+    x = workloads.normal_bf16(5, 1, 0, T * H).reshape(T, H)
+    w = np.zeros((H, E), dtype=np.uint16)
+    s, i, L = run_ws(x, w, k, logits=True)
+    assert np.all(L == 0.0)
+    assert np.array_equal(i, np.tile(np.arange(k, dtype=np.int32), (T, 1)))
+    assert np.all(np.abs(s - 1.0 / k) <= 1e-7)
+
+
+@pytest.mark.parametrize("T,E", [(1, 16), (4, 32), (2, 24)])
+def test_k_equals_E_full_softmax(T, E):
+    """k = E: every expert is selected, in logit order; the scores are the softmax
+    over all E logits."""
+    wl = workloads.RouterWorkload(f"few_kE_{T}_{E}", T, 1024, E, E, seed=40 + E)
+    s, i, L = run_ws(wl.hidden(), wl.gate_weight(), E, logits=True)
+    ref = oracle.fused_topk_gating(wl.hidden(), wl.gate_weight(), E, want_logits=True)
+    parity.check(s, i, ref, label=wl.name)
+    assert np.array_equal(np.sort(i, axis=1), np.tile(np.arange(E, dtype=np.int32), (T, 1)))
