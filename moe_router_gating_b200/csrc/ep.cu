@@ -42,9 +42,19 @@ int current_sms() {
   return n;
 }
 
+// Combine: as many CTAs as the SMs hold at once (every warp resident, each
+// looping over the row parts), or fewer when there are fewer items.
 template <int KMAX>
-tk_status launch_combine(const tkg::EpCombineParams& p, int grid, cudaStream_t s) {
-  tkg::ep_combine_kernel<KMAX><<<grid, tkg::EP_THREADS, 0, s>>>(p);
+tk_status launch_combine(const tkg::EpCombineParams& p, int num_sms, cudaStream_t s) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tkg::ep_combine_kernel<KMAX>, tkg::EP_THREADS, 0) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return TK_ERR_CUDA;
+  const int64_t warps_per_cta = tkg::EP_THREADS / 32;
+  int64_t grid = (p.T * p.parts + warps_per_cta - 1) / warps_per_cta;
+  if (grid > static_cast<int64_t>(num_sms) * per_sm) grid = static_cast<int64_t>(num_sms) * per_sm;
+  tkg::ep_combine_kernel<KMAX><<<static_cast<int>(grid < 1 ? 1 : grid), tkg::EP_THREADS, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? TK_OK : TK_ERR_CUDA;
 }
 
@@ -124,14 +134,16 @@ tk_status tk_gating_fused_combine(const uint64_t* rows, int64_t T, int64_t H, in
   p.err_word = err;
   p.T = T;
   p.vec_per_row = H / 8;
+  p.parts = static_cast<int32_t>((p.vec_per_row + tkg::EP_PART_VECS - 1) / tkg::EP_PART_VECS);
+  p.part_vecs = (p.vec_per_row + p.parts - 1) / p.parts;
+  if (p.parts > 1) p.part_vecs = (p.part_vecs + 31) / 32 * 32;  // whole lane rounds; the last part shorter
   p.k = k;
   p.E = E;
-  const int grid = ep_grid(T, sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (k <= 4) return launch_combine<4>(p, grid, s);
-  if (k <= 8) return launch_combine<8>(p, grid, s);
-  if (k <= 16) return launch_combine<16>(p, grid, s);
-  return launch_combine<32>(p, grid, s);
+  if (k <= 4) return launch_combine<4>(p, sms, s);
+  if (k <= 8) return launch_combine<8>(p, sms, s);
+  if (k <= 16) return launch_combine<16>(p, sms, s);
+  return launch_combine<32>(p, sms, s);
 }
 
 tk_status tk_gating_ep_rows_table(const int32_t* offsets_all, int32_t R, int32_t E, int32_t rank, const uint64_t* bases,

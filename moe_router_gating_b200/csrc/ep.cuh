@@ -49,9 +49,15 @@ struct EpCombineParams {
   uint32_t* err_word;
   int64_t T;
   int64_t vec_per_row;
+  int64_t part_vecs;  // 16-byte vectors of a row part (a multiple of 32, or the whole row)
+  int32_t parts;      // parts per row: a warp combines one part of one token's row at a time
   int32_t k;
   int32_t E;
 };
+
+// Row parts of about 224 vectors (seven per lane): enough work items to spread
+// a few thousand tokens evenly over every resident warp.
+constexpr int64_t EP_PART_VECS = 224;
 
 constexpr uint32_t EP_ERR_ROW = 1u << 8;
 
@@ -119,15 +125,20 @@ __device__ __forceinline__ uint32_t ep_pack_bf16x2(float lo, float hi) {
   return l | (h << 16);
 }
 
-// One warp per token (grid-stride): out[t] = sum_{j < k} scores[t, j] * row(t, j),
-// fp32 fused multiply-adds in rank order j = 0 .. k-1, rounded once to bf16.
-// Lane j < k looks up assignment j's row address; the warp reads them by shuffle.
+// One warp per part of a token's row (grid-stride over T x parts work items):
+// out[t] = sum_{j < k} scores[t, j] * row(t, j), fp32 fused multiply-adds in
+// rank order j = 0 .. k-1, rounded once to bf16.  Lane j < k looks up
+// assignment j's row address; the warp reads them by shuffle.
 template <int KMAX>
 __global__ void __launch_bounds__(EP_THREADS) ep_combine_kernel(const EpCombineParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * EP_THREADS + threadIdx.x) >> 5;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (EP_THREADS / 32);
-  for (int64_t t = warp; t < p.T; t += warps) {
+  const int64_t items = p.T * p.parts;
+  for (int64_t item = warp; item < items; item += warps) {
+    const int64_t t = item / p.parts;
+    const int64_t v0 = (item - t * p.parts) * p.part_vecs;
+    const int64_t v1 = v0 + p.part_vecs < p.vec_per_row ? v0 + p.part_vecs : p.vec_per_row;
     uint64_t my_row = 0;
     float my_w = 0.0f;
     if (lane < p.k) {
@@ -154,7 +165,7 @@ __global__ void __launch_bounds__(EP_THREADS) ep_combine_kernel(const EpCombineP
       w[j] = __shfl_sync(0xffffffffu, my_w, j);
     }
     uint4* dst = p.out + t * p.vec_per_row;
-    for (int64_t v = lane; v < p.vec_per_row; v += 32) {
+    for (int64_t v = v0 + lane; v < v1; v += 32) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       constexpr int G = KMAX < 8 ? KMAX : 8;  // rows loaded before their multiply-adds
 #pragma unroll

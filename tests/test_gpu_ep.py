@@ -130,6 +130,7 @@ def run_case(R, T, H, k, E, seed, kind="uniform"):
     (4, (100, 1, 0, 333), 128, 3, 32, "uniform"),
     (8, (64,) * 8, 7168, 8, 256, "uniform"),
     (2, (2000, 1500), 1024, 32, 64, "skew"),
+    (1, (513,), 3592, 8, 64, "uniform"),   # combine rows in three parts, the last one shorter
 ])
 def test_emulated_ranks_match_the_oracle(R, T, H, k, E, kind):
     run_case(R, T, H, k, E, seed=R * 7 + k, kind=kind)
