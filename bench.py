@@ -903,7 +903,7 @@ def run_ep_ours(args, wl):
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
 
     def dispatch():
-        ep.dispatch_rows(x, ids, offsets, sorted_slots, rows, E, stream)
+        ep.dispatch_rows(x, ids, offsets, slot_pos, rows, E, stream)
 
     def combine():
         ep.combine_rows(out_rows, ids, offsets, slot_pos, scores, out, E, stream)
@@ -928,7 +928,7 @@ def run_ep_ours(args, wl):
     if tk.device_error(clear=True):
         raise SystemExit("an expert-parallel kernel reported a bad row address")
     placed = T * k
-    d_bytes = 2 * (2 * H) * placed            # each placed row read once (from L2 when repeated) and written once
+    d_bytes = 2 * H * T + (2 * H) * placed    # each token row read once, each placed row written once
     c_bytes = (2 * H) * placed + 2 * H * T + 12 * T * k   # k rows read per token, one row written, metadata
     peaks, peak_src = load_peaks()
     ms = t_d + t_c

@@ -538,14 +538,16 @@ TK_API tk_status tk_gating_route_static(const int32_t* ids, int64_t T, int32_t k
 
 /*
  * tk_gating_fused_dispatch -- copy every placed assignment's token row to
- * its row in the expert buffer.
+ * its row in the expert buffer.  Each token row is read once and stored to
+ * each of its k destination rows.
  *
  *   tokens        device, bf16 [T, H] row-major, 16-byte aligned.
  *   T, H, k, E    tokens (T >= 0), hidden size (H % 8 == 0), experts per
  *                 token (1 <= k <= 32), experts (1 <= E <= 1024); T*k < 2^31.
  *   ids           device, int32 [T, k]: the experts (tk_gating_fused_topk).
  *   offsets       device, int32 [E + 1]     } tk_gating_route of ids
- *   sorted_slots  device, int32 [T * k]     }
+ *   slot_pos      device, int32 [T, k]      }   (assignments whose id is
+ *                 outside [0, E) or whose slot_pos is -1 are not copied)
  *   rows          device, uint64 [E]: destination address of expert e's first
  *                 row for this rank (16-byte aligned; device or peer memory).
  *   stream        cudaStream_t (void*), may be NULL.
@@ -557,7 +559,7 @@ TK_API tk_status tk_gating_route_static(const int32_t* ids, int64_t T, int32_t k
  * T == 0 returns TK_OK and launches nothing.
  */
 TK_API tk_status tk_gating_fused_dispatch(const void* tokens, int64_t T, int64_t H, int32_t k, int32_t E,
-                                          const int32_t* ids, const int32_t* offsets, const int32_t* sorted_slots,
+                                          const int32_t* ids, const int32_t* offsets, const int32_t* slot_pos,
                                           const uint64_t* rows, void* stream);
 
 /*

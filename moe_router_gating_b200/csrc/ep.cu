@@ -27,14 +27,6 @@ tk_status validate_ep(int64_t T, int64_t H, int32_t k, int32_t E) {
   return TK_OK;
 }
 
-int ep_grid(int64_t items_per_warp_total, int num_sms) {
-  const int64_t warps_per_cta = tkg::EP_THREADS / 32;
-  int64_t g = (items_per_warp_total + warps_per_cta - 1) / warps_per_cta;
-  const int64_t cap = static_cast<int64_t>(num_sms) * 4;
-  if (g > cap) g = cap;
-  return static_cast<int>(g < 1 ? 1 : g);
-}
-
 int current_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -42,19 +34,43 @@ int current_sms() {
   return n;
 }
 
-// Combine: as many CTAs as the SMs hold at once (every warp resident, each
-// looping over the row parts), or fewer when there are fewer items.
+// As many CTAs as the SMs hold at once (every warp resident, each looping over
+// the work items), or fewer when there are fewer items (one per warp).
+template <typename Kernel>
+int resident_grid(Kernel kernel, int64_t items, int num_sms) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, tkg::EP_THREADS, 0) != cudaSuccess || per_sm < 1)
+    return 0;
+  const int64_t warps_per_cta = tkg::EP_THREADS / 32;
+  int64_t grid = (items + warps_per_cta - 1) / warps_per_cta;
+  if (grid > static_cast<int64_t>(num_sms) * per_sm) grid = static_cast<int64_t>(num_sms) * per_sm;
+  return static_cast<int>(grid < 1 ? 1 : grid);
+}
+
+// Row parts of about EP_PART_VECS vectors: parts per row and vectors per part
+// (a multiple of 32 when the row has several parts; the last part shorter).
+// A part never exceeds EP_PART_VECS (a multiple of 32), so a lane holds at most
+// EP_LANE_VECS vectors of it.
+bool row_parts(int64_t vec_per_row, int32_t* parts, int64_t* part_vecs) {
+  *parts = static_cast<int32_t>((vec_per_row + tkg::EP_PART_VECS - 1) / tkg::EP_PART_VECS);
+  *part_vecs = (vec_per_row + *parts - 1) / *parts;
+  if (*parts > 1) *part_vecs = (*part_vecs + 31) / 32 * 32;
+  return *part_vecs <= tkg::EP_PART_VECS && static_cast<int64_t>(*parts) * *part_vecs >= vec_per_row;
+}
+
 template <int KMAX>
 tk_status launch_combine(const tkg::EpCombineParams& p, int num_sms, cudaStream_t s) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tkg::ep_combine_kernel<KMAX>, tkg::EP_THREADS, 0) !=
-          cudaSuccess ||
-      per_sm < 1)
-    return TK_ERR_CUDA;
-  const int64_t warps_per_cta = tkg::EP_THREADS / 32;
-  int64_t grid = (p.T * p.parts + warps_per_cta - 1) / warps_per_cta;
-  if (grid > static_cast<int64_t>(num_sms) * per_sm) grid = static_cast<int64_t>(num_sms) * per_sm;
-  tkg::ep_combine_kernel<KMAX><<<static_cast<int>(grid < 1 ? 1 : grid), tkg::EP_THREADS, 0, s>>>(p);
+  const int grid = resident_grid(tkg::ep_combine_kernel<KMAX>, p.T * p.parts, num_sms);
+  if (grid == 0) return TK_ERR_CUDA;
+  tkg::ep_combine_kernel<KMAX><<<grid, tkg::EP_THREADS, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TK_OK : TK_ERR_CUDA;
+}
+
+template <int KMAX>
+tk_status launch_dispatch(const tkg::EpDispatchParams& p, int num_sms, cudaStream_t s) {
+  const int grid = resident_grid(tkg::ep_dispatch_kernel<KMAX>, p.T * p.parts, num_sms);
+  if (grid == 0) return TK_ERR_CUDA;
+  tkg::ep_dispatch_kernel<KMAX><<<grid, tkg::EP_THREADS, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? TK_OK : TK_ERR_CUDA;
 }
 
@@ -85,14 +101,13 @@ static_assert(sizeof(IpcHandle) <= TK_EP_IPC_HANDLE_BYTES, "handle size");
 extern "C" {
 
 tk_status tk_gating_fused_dispatch(const void* tokens, int64_t T, int64_t H, int32_t k, int32_t E, const int32_t* ids,
-                                   const int32_t* offsets, const int32_t* sorted_slots, const uint64_t* rows,
+                                   const int32_t* offsets, const int32_t* slot_pos, const uint64_t* rows,
                                    void* stream) {
   tk_status st = validate_ep(T, H, k, E);
   if (st != TK_OK) return st;
   if (T == 0) return TK_OK;
-  if (!tokens || !ids || !offsets || !sorted_slots || !rows) return TK_ERR_INVALID_ARG;
-  if (!aligned(tokens, 16) || !aligned(ids, 4) || !aligned(offsets, 4) || !aligned(sorted_slots, 4) ||
-      !aligned(rows, 8))
+  if (!tokens || !ids || !offsets || !slot_pos || !rows) return TK_ERR_INVALID_ARG;
+  if (!aligned(tokens, 16) || !aligned(ids, 4) || !aligned(offsets, 4) || !aligned(slot_pos, 4) || !aligned(rows, 8))
     return TK_ERR_ALIGNMENT;
   uint32_t* err = tkg::device_error_word();
   const int sms = current_sms();
@@ -101,14 +116,19 @@ tk_status tk_gating_fused_dispatch(const void* tokens, int64_t T, int64_t H, int
   p.tokens = static_cast<const uint4*>(tokens);
   p.ids = ids;
   p.offsets = offsets;
-  p.sorted_slots = sorted_slots;
+  p.slot_pos = slot_pos;
   p.rows = rows;
   p.err_word = err;
+  p.T = T;
   p.vec_per_row = H / 8;
+  if (!row_parts(p.vec_per_row, &p.parts, &p.part_vecs)) return TK_ERR_UNSUPPORTED;
   p.k = k;
   p.E = E;
-  tkg::ep_dispatch_kernel<<<ep_grid(T * k, sms), tkg::EP_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(p);
-  return cudaGetLastError() == cudaSuccess ? TK_OK : TK_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k <= 4) return launch_dispatch<4>(p, sms, s);
+  if (k <= 8) return launch_dispatch<8>(p, sms, s);
+  if (k <= 16) return launch_dispatch<16>(p, sms, s);
+  return launch_dispatch<32>(p, sms, s);
 }
 
 tk_status tk_gating_fused_combine(const uint64_t* rows, int64_t T, int64_t H, int32_t k, int32_t E, const int32_t* ids,
@@ -134,9 +154,7 @@ tk_status tk_gating_fused_combine(const uint64_t* rows, int64_t T, int64_t H, in
   p.err_word = err;
   p.T = T;
   p.vec_per_row = H / 8;
-  p.parts = static_cast<int32_t>((p.vec_per_row + tkg::EP_PART_VECS - 1) / tkg::EP_PART_VECS);
-  p.part_vecs = (p.vec_per_row + p.parts - 1) / p.parts;
-  if (p.parts > 1) p.part_vecs = (p.part_vecs + 31) / 32 * 32;  // whole lane rounds; the last part shorter
+  if (!row_parts(p.vec_per_row, &p.parts, &p.part_vecs)) return TK_ERR_UNSUPPORTED;
   p.k = k;
   p.E = E;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

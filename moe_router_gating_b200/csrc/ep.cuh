@@ -13,9 +13,11 @@
 // all-to-all runs.  Plain 16-byte loads and stores; no multicast.
 //
 // Assignment s = t*k + j (token t, rank j) with expert e = ids[s] sits at
-// position p = slot_pos[s] of this rank's expert-grouped order (offsets,
-// sorted_slots, slot_pos from tk_gating_route); its row in the expert buffer
-// is rows[e] + (p - offsets[e]).
+// position p = slot_pos[s] of this rank's expert-grouped order (offsets and
+// slot_pos from tk_gating_route); its row in the expert buffer is
+// rows[e] + (p - offsets[e]).  Both kernels work token by token, a warp per
+// part of a token's row (EP_PART_VECS 16-byte vectors), over as many CTAs as
+// the SMs hold at once.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,16 +27,18 @@
 namespace tkg {
 
 constexpr int EP_THREADS = 256;  // 8 warps; a warp moves one row at a time
-constexpr int EP_UNROLL = 4;     // 16-byte vectors in flight per lane
 
 struct EpDispatchParams {
   const uint4* tokens;          // [T, H] bf16, rows of vec_per_row 16-byte vectors
   const int32_t* ids;           // [T * k]
   const int32_t* offsets;       // [E + 1]
-  const int32_t* sorted_slots;  // [T * k]
+  const int32_t* slot_pos;      // [T * k]
   const uint64_t* rows;         // [E] destination address of expert e's first row
   uint32_t* err_word;           // bit EP_ERR_ROW: a row address was not 16-byte aligned
+  int64_t T;
   int64_t vec_per_row;          // H / 8
+  int64_t part_vecs;            // 16-byte vectors of a row part (a multiple of 32, or the whole row)
+  int32_t parts;                // parts per row
   int32_t k;
   int32_t E;
 };
@@ -58,6 +62,7 @@ struct EpCombineParams {
 // Row parts of about 224 vectors (seven per lane): enough work items to spread
 // a few thousand tokens evenly over every resident warp.
 constexpr int64_t EP_PART_VECS = 224;
+constexpr int EP_LANE_VECS = static_cast<int>(EP_PART_VECS / 32);  // a lane's vectors of one part, at most
 
 constexpr uint32_t EP_ERR_ROW = 1u << 8;
 
@@ -75,35 +80,60 @@ __device__ __forceinline__ uint4 ep_ld(const uint4* p) {
   return v;
 }
 
-// One warp per placed position p (grid-stride): copy token sorted_slots[p] / k
-// to its row in the destination buffer of expert ids[sorted_slots[p]].
+// Row address of assignment s = t*k + lane for lane < k (0: nothing there --
+// an id outside [0, E), slot_pos -1, a position outside its expert's range, or
+// a row address that is not 16-byte aligned, which is also reported).
+__device__ __forceinline__ uint64_t ep_row_of(const uint64_t* rows, const int32_t* ids, const int32_t* offsets,
+                                              const int32_t* slot_pos, int64_t s, int32_t E, int64_t vec_per_row,
+                                              uint32_t* err_word) {
+  const int32_t e = __ldg(ids + s);
+  const int32_t pos = __ldg(slot_pos + s);
+  if (static_cast<uint32_t>(e) >= static_cast<uint32_t>(E) || pos < 0) return 0;
+  const int32_t o0 = __ldg(offsets + e), o1 = __ldg(offsets + e + 1);
+  const uint64_t base = __ldg(rows + e);
+  if (pos < o0 || pos >= o1) return 0;
+  if (base & 15u) {
+    atomicOr(err_word, EP_ERR_ROW);
+    return 0;
+  }
+  return base + static_cast<uint64_t>(pos - o0) * static_cast<uint64_t>(vec_per_row) * 16u;
+}
+
+// One warp per part of a token's row (grid-stride over T x parts work items):
+// the token's vectors are loaded once and stored to each of its k destination
+// rows (this rank's buffers or peers'), so a token row crosses from memory once
+// however many experts it goes to.  Lane j < k looks up assignment j's row; the
+// warp reads the addresses by shuffle.
+template <int KMAX>
 __global__ void __launch_bounds__(EP_THREADS) ep_dispatch_kernel(const EpDispatchParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * EP_THREADS + threadIdx.x) >> 5;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (EP_THREADS / 32);
-  const int64_t placed = __ldg(p.offsets + p.E);
-  for (int64_t pos = warp; pos < placed; pos += warps) {
-    const int32_t s = __ldg(p.sorted_slots + pos);
-    const int32_t e = __ldg(p.ids + s);
-    if (static_cast<uint32_t>(e) >= static_cast<uint32_t>(p.E)) continue;  // not produced by the routing
-    const int32_t o0 = __ldg(p.offsets + e), o1 = __ldg(p.offsets + e + 1);
-    if (pos < o0 || pos >= o1) continue;
-    const uint64_t base = __ldg(p.rows + e);
-    if (base & 15u) {
-      if (lane == 0) atomicOr(p.err_word, EP_ERR_ROW);
-      continue;
-    }
-    const uint4* src = p.tokens + static_cast<int64_t>(s / p.k) * p.vec_per_row;
-    uint4* dst = reinterpret_cast<uint4*>(base) + (pos - o0) * p.vec_per_row;
-    int64_t v = lane;
-    for (; v + 32 * (EP_UNROLL - 1) < p.vec_per_row; v += 32 * EP_UNROLL) {
-      uint4 r[EP_UNROLL];
+  const int64_t items = p.T * p.parts;
+  for (int64_t item = warp; item < items; item += warps) {
+    const int64_t t = item / p.parts;
+    const int64_t v0 = (item - t * p.parts) * p.part_vecs;
+    const int64_t v1 = v0 + p.part_vecs < p.vec_per_row ? v0 + p.part_vecs : p.vec_per_row;
+    const uint64_t my_row =
+        lane < p.k ? ep_row_of(p.rows, p.ids, p.offsets, p.slot_pos, t * p.k + lane, p.E, p.vec_per_row, p.err_word)
+                   : 0;
+    uint64_t row[KMAX];
 #pragma unroll
-      for (int u = 0; u < EP_UNROLL; ++u) r[u] = ep_ld_nc(src + v + 32 * u);
+    for (int j = 0; j < KMAX; ++j) row[j] = __shfl_sync(0xffffffffu, my_row, j);
+    // all of this lane's vectors of the part in flight at once, then each stored k times
+    const uint4* src = p.tokens + t * p.vec_per_row;
+    uint4 x[EP_LANE_VECS];
 #pragma unroll
-      for (int u = 0; u < EP_UNROLL; ++u) dst[v + 32 * u] = r[u];
-    }
-    for (; v < p.vec_per_row; v += 32) dst[v] = ep_ld_nc(src + v);
+    for (int u = 0; u < EP_LANE_VECS; ++u)
+      if (v0 + lane + 32 * u < v1) x[u] = ep_ld_nc(src + v0 + lane + 32 * u);
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < p.k && row[j] != 0) {
+        uint4* dst = reinterpret_cast<uint4*>(row[j]) + v0 + lane;
+#pragma unroll
+        for (int u = 0; u < EP_LANE_VECS; ++u)
+          if (v0 + lane + 32 * u < v1) dst[32 * u] = x[u];
+      }
   }
   // the stores (possibly to another GPU) are ordered before whatever the host
   // orders after this kernel
@@ -143,19 +173,8 @@ __global__ void __launch_bounds__(EP_THREADS) ep_combine_kernel(const EpCombineP
     float my_w = 0.0f;
     if (lane < p.k) {
       const int64_t s = t * p.k + lane;
-      const int32_t e = __ldg(p.ids + s);
-      const int32_t pos = __ldg(p.slot_pos + s);
-      if (static_cast<uint32_t>(e) < static_cast<uint32_t>(p.E) && pos >= 0) {
-        const int32_t o0 = __ldg(p.offsets + e), o1 = __ldg(p.offsets + e + 1);
-        const uint64_t base = __ldg(p.rows + e);
-        if (pos >= o0 && pos < o1) {
-          if (base & 15u)
-            atomicOr(p.err_word, EP_ERR_ROW);
-          else
-            my_row = base + static_cast<uint64_t>(pos - o0) * static_cast<uint64_t>(p.vec_per_row) * 16u;
-        }
-        my_w = __ldg(p.scores + s);
-      }
+      my_row = ep_row_of(p.rows, p.ids, p.offsets, p.slot_pos, s, p.E, p.vec_per_row, p.err_word);
+      my_w = __ldg(p.scores + s);
     }
     uint64_t row[KMAX];
     float w[KMAX];
@@ -165,21 +184,33 @@ __global__ void __launch_bounds__(EP_THREADS) ep_combine_kernel(const EpCombineP
       w[j] = __shfl_sync(0xffffffffu, my_w, j);
     }
     uint4* dst = p.out + t * p.vec_per_row;
-    for (int64_t v = v0 + lane; v < v1; v += 32) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // two of the lane's vectors per step: up to 2 x 8 row loads in flight
+    for (int64_t v = v0 + lane; v < v1; v += 64) {
+      const bool two = v + 32 < v1;
+      float acc[2][8] = {{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}};
       constexpr int G = KMAX < 8 ? KMAX : 8;  // rows loaded before their multiply-adds
 #pragma unroll
       for (int j0 = 0; j0 < KMAX; j0 += G) {
-        uint4 y[G];
+        uint4 y[2][G];
 #pragma unroll
         for (int u = 0; u < G; ++u)
-          if (j0 + u < p.k && row[j0 + u] != 0) y[u] = ep_ld(reinterpret_cast<const uint4*>(row[j0 + u]) + v);
+          if (j0 + u < p.k && row[j0 + u] != 0) {
+            const uint4* r = reinterpret_cast<const uint4*>(row[j0 + u]);
+            y[0][u] = ep_ld(r + v);
+            if (two) y[1][u] = ep_ld(r + v + 32);
+          }
 #pragma unroll
         for (int u = 0; u < G; ++u)
-          if (j0 + u < p.k && row[j0 + u] != 0) ep_fma8(acc, w[j0 + u], y[u]);
+          if (j0 + u < p.k && row[j0 + u] != 0) {
+            ep_fma8(acc[0], w[j0 + u], y[0][u]);
+            if (two) ep_fma8(acc[1], w[j0 + u], y[1][u]);
+          }
       }
-      dst[v] = make_uint4(ep_pack_bf16x2(acc[0], acc[1]), ep_pack_bf16x2(acc[2], acc[3]),
-                          ep_pack_bf16x2(acc[4], acc[5]), ep_pack_bf16x2(acc[6], acc[7]));
+      dst[v] = make_uint4(ep_pack_bf16x2(acc[0][0], acc[0][1]), ep_pack_bf16x2(acc[0][2], acc[0][3]),
+                          ep_pack_bf16x2(acc[0][4], acc[0][5]), ep_pack_bf16x2(acc[0][6], acc[0][7]));
+      if (two)
+        dst[v + 32] = make_uint4(ep_pack_bf16x2(acc[1][0], acc[1][1]), ep_pack_bf16x2(acc[1][2], acc[1][3]),
+                                 ep_pack_bf16x2(acc[1][4], acc[1][5]), ep_pack_bf16x2(acc[1][6], acc[1][7]));
     }
   }
 }

@@ -125,13 +125,14 @@ def _stream(stream, device) -> int:
     return int((stream or torch.cuda.current_stream(device)).cuda_stream)
 
 
-def dispatch_rows(tokens, ids, offsets, sorted_slots, rows, num_experts: int, stream=None) -> None:
-    """Raw dispatch with a row-address table ``rows`` (uint64 [E] on the device)."""
+def dispatch_rows(tokens, ids, offsets, slot_pos, rows, num_experts: int, stream=None) -> None:
+    """Raw dispatch with a row-address table ``rows`` (uint64 [E] on the device);
+    ``offsets`` and ``slot_pos`` are tk_gating_route's for ``ids``."""
     T, H = tokens.shape
     k = ids.shape[1]
     with _device(tokens):
         _check(_lib().tk_gating_fused_dispatch(tokens.data_ptr(), T, H, k, int(num_experts), ids.data_ptr(),
-                                               offsets.data_ptr(), sorted_slots.data_ptr(), rows.data_ptr(),
+                                               offsets.data_ptr(), slot_pos.data_ptr(), rows.data_ptr(),
                                                _stream(stream, tokens.device)), "tk_gating_fused_dispatch")
 
 
@@ -301,7 +302,7 @@ class ExpertParallelGroup:
         recv_rows = check_capacities(offsets_all.cpu().tolist(), self.capacities)[self.rank]
         rows, out_rows, recv_offsets = rows_table(offsets_all, self.rank, self.bases, self.out_bases, self.H, stream)
         self._barrier(stream)  # every receive buffer is free
-        dispatch_rows(tokens, expert_ids, offsets, sorted_slots, rows, self.E, stream)
+        dispatch_rows(tokens, expert_ids, offsets, slot_pos, rows, self.E, stream)
         self._barrier(stream)  # every rank's rows have landed
         return self.recv[:recv_rows], DispatchHandle(expert_ids, offsets, slot_pos, out_rows, recv_offsets, recv_rows)
 

@@ -98,7 +98,7 @@ def run_case(R, T, H, k, E, seed, kind="uniform"):
             assert int(orows[e]) == int(out_list[q]) + plan.dest_row[e] * 2 * H, (s, e)
     for s in range(R):  # every source rank's dispatch writes into every receive buffer
         x = bf16_bits_to_torch(toks[s]).to(dev)
-        ep.dispatch_rows(x, d_ids[s], routes[s][0], routes[s][1], tables[s][0], E)
+        ep.dispatch_rows(x, d_ids[s], routes[s][0], routes[s][2], tables[s][0], E)
     torch.cuda.synchronize()
     per = E // R
     for q in range(R):
@@ -167,7 +167,7 @@ def test_misaligned_row_address_is_reported_not_written():
     buf = torch.zeros(T * k * H + 64, dtype=torch.bfloat16, device=dev)
     rows = torch.tensor([buf.data_ptr() + 2] * E, dtype=torch.uint64, device=dev)  # 2 bytes off alignment
     tk.device_error(clear=True)
-    ep.dispatch_rows(x, ids, offsets, sorted_slots, rows, E)
+    ep.dispatch_rows(x, ids, offsets, slot_pos, rows, E)
     torch.cuda.synchronize()
     assert tk.device_error(clear=True) & (1 << 8)
     assert torch.count_nonzero(buf) == 0
