@@ -524,9 +524,8 @@ TK_API tk_status tk_gating_route_static(const int32_t* ids, int64_t T, int32_t k
  * addresses: rows[e] = the address of this source rank's first row for
  * expert e in the buffer of the rank that holds e (a local buffer, or another
  * GPU's buffer opened with tk_gating_ep_ipc_open).  Assignment s with expert
- * e = ids[s] at position p = slot_pos[s] of the expert-grouped order (offsets,
- * sorted_slots, slot_pos from tk_gating_route) uses row rows[e] + (p -
- * offsets[e]).  Dispatch stores each token row there; combine loads the
+ * e = ids[s] at position p = slot_pos[s] of the expert-grouped order (offsets
+ * and slot_pos from tk_gating_route) uses row rows[e] + (p - offsets[e]).  Dispatch stores each token row there; combine loads the
  * expert output rows from there (the receiver pulls, as the page's section 6
  * recommends), so the data crosses NVLink once and no all-to-all runs.
  * Ordering between ranks is the caller's: every rank's dispatch has to be
